@@ -1,0 +1,189 @@
+"""fp64 CPU oracle for the Spark FFN and statistical top-k.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this package.  The product
+library never links or calls it, and it imports nothing from the product.
+
+The arithmetic lives in ``spark_oracle.c`` (plain loops in double precision);
+this module only compiles it with gcc and marshals numpy arrays through ctypes.
+Source of the method: the paper-notes page "Spark Transformer: Reactivating
+Sparsity in FFN and Attention", section 方法详解/关键设计 ("Spark FFN" and
+"Statistical Top-k").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "spark_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libspark_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GELU_TANH = 0
+GELU_ERF = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile spark_oracle.c into libspark_oracle.so (gcc, OpenMP, no FMA contraction)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-D_GNU_SOURCE", "-ffp-contract=off", "-fno-fast-math",
+           "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        # SPARK_ORACLE_LIB lets the mutation test load a deliberately broken copy.
+        lib = ctypes.CDLL(os.environ.get("SPARK_ORACLE_LIB") or build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_bf16_to_f64.restype = ctypes.c_double
+        lib.oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_normal_upper_tail.restype = ctypes.c_double
+        lib.oracle_normal_upper_tail.argtypes = [ctypes.c_double]
+        lib.oracle_topk_quantile.restype = ctypes.c_double
+        lib.oracle_topk_quantile.argtypes = [ctypes.c_double, ctypes.c_double]
+        lib.oracle_row_stats.restype = None
+        lib.oracle_row_stats.argtypes = [dp, ctypes.c_long, dp, dp]
+        lib.oracle_theta.restype = ctypes.c_double
+        lib.oracle_theta.argtypes = [dp, ctypes.c_long, ctypes.c_long, dp, dp]
+        lib.oracle_gelu_tanh.restype = ctypes.c_double
+        lib.oracle_gelu_tanh.argtypes = [ctypes.c_double]
+        lib.oracle_gelu_erf.restype = ctypes.c_double
+        lib.oracle_gelu_erf.argtypes = [ctypes.c_double]
+        lib.oracle_stat_topk.restype = ctypes.c_int
+        lib.oracle_stat_topk.argtypes = [ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_long,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_spark_ffn.restype = ctypes.c_int
+        lib.oracle_spark_ffn.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_long] * 5 + [
+            ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_rmsnorm.restype = None
+        lib.oracle_rmsnorm.argtypes = [dp, ctypes.c_long, ctypes.c_double, dp]
+        lib.oracle_num_threads_available.restype = ctypes.c_int
+        lib.oracle_num_threads_available.argtypes = []
+        _lib = lib
+        return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dptr(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def max_threads() -> int:
+    return int(_load().oracle_num_threads_available())
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float64, one element at a time."""
+    lib = _load()
+    flat = np.ascontiguousarray(bits, dtype=np.uint16).ravel()
+    return np.array([lib.oracle_bf16_to_f64(int(b)) for b in flat], dtype=np.float64).reshape(bits.shape)
+
+
+def topk_quantile(k: float, d: float) -> float:
+    """Q(1 - k/d), the standard-normal quantile, by bisection on erfc."""
+    return float(_load().oracle_topk_quantile(float(k), float(d)))
+
+
+def normal_upper_tail(z: float) -> float:
+    return float(_load().oracle_normal_upper_tail(float(z)))
+
+
+def row_stats(x: np.ndarray) -> tuple[float, float]:
+    """Population mean and std of a 1-D row (two passes, fp64)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    m = ctypes.c_double()
+    s = ctypes.c_double()
+    _load().oracle_row_stats(_dptr(x), x.size, ctypes.byref(m), ctypes.byref(s))
+    return m.value, s.value
+
+
+def theta(x: np.ndarray, k: int) -> float:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    return float(_load().oracle_theta(_dptr(x), x.size, int(k), None, None))
+
+
+def gelu(s: float, kind: int = GELU_TANH) -> float:
+    lib = _load()
+    return float(lib.oracle_gelu_erf(s) if kind == GELU_ERF else lib.oracle_gelu_tanh(s))
+
+
+def stat_topk(x: np.ndarray, k: int, n_threads: int = 1):
+    """Statistical top-k + soft threshold on fp32 rows [rows, d].
+
+    Returns (out fp64 [rows,d], theta [rows], mean [rows], std [rows]).
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim == 1:
+        x = x[None, :]
+    rows, d = x.shape
+    out = np.empty((rows, d), dtype=np.float64)
+    th = np.empty(rows, dtype=np.float64)
+    mu = np.empty(rows, dtype=np.float64)
+    sd = np.empty(rows, dtype=np.float64)
+    rc = _load().oracle_stat_topk(_ptr(x), rows, d, int(k), _ptr(out), _ptr(th), _ptr(mu),
+                                  _ptr(sd), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_stat_topk: invalid arguments (d={d}, k={k})")
+    return out, th, mu, sd
+
+
+def spark_ffn(q_bits, K1_bits, K2_bits, V_bits, r: int, k: int, gelu_kind: int = GELU_TANH,
+              override_active=None, n_threads: int = 1):
+    """Spark FFN forward on bf16 bit patterns (uint16 arrays).
+
+    q_bits [T, d_model], K1_bits [d_ff, r], K2_bits [d_ff, d_model - r],
+    V_bits [d_ff, d_model].  Returns a dict with out [T, d_model] (fp64),
+    x [T, d_ff], theta/mean/std [T] and active [T, d_ff] (bool, x > theta).
+    """
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    if q.ndim == 1:
+        q = q[None, :]
+    K1 = np.ascontiguousarray(K1_bits, dtype=np.uint16)
+    K2 = np.ascontiguousarray(K2_bits, dtype=np.uint16)
+    V = np.ascontiguousarray(V_bits, dtype=np.uint16)
+    T, d_model = q.shape
+    d_ff = K1.shape[0]
+    if K1.shape != (d_ff, r) or K2.shape != (d_ff, d_model - r) or V.shape != (d_ff, d_model):
+        raise ValueError("oracle.spark_ffn: inconsistent shapes")
+    ov = None
+    if override_active is not None:
+        ov = np.ascontiguousarray(override_active, dtype=np.uint8).reshape(T, d_ff)
+    out = np.empty((T, d_model), dtype=np.float64)
+    x = np.empty((T, d_ff), dtype=np.float64)
+    th = np.empty(T, dtype=np.float64)
+    mu = np.empty(T, dtype=np.float64)
+    sd = np.empty(T, dtype=np.float64)
+    act = np.empty((T, d_ff), dtype=np.uint8)
+    rc = _load().oracle_spark_ffn(_ptr(q), _ptr(K1), _ptr(K2), _ptr(V), T, d_model, r, d_ff, int(k),
+                                  int(gelu_kind), _ptr(ov), _ptr(out), _ptr(x), _ptr(th), _ptr(mu),
+                                  _ptr(sd), _ptr(act), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_spark_ffn: invalid arguments")
+    return {"out": out, "x": x, "theta": th, "mean": mu, "std": sd, "active": act.astype(bool)}
+
+
+def rmsnorm(h: np.ndarray, eps: float = 1e-6) -> np.ndarray:
+    h = np.ascontiguousarray(h, dtype=np.float64)
+    y = np.empty_like(h)
+    _load().oracle_rmsnorm(_dptr(h), h.size, float(eps), _dptr(y))
+    return y
