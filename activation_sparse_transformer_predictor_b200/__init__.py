@@ -1,1 +1,126 @@
-"""Spark FFN with statistical top-k on B200 (sm_100a)."""
+"""Spark FFN with statistical top-k on NVIDIA B200 (sm_100a).
+
+Public Python API over the C ABI of ``libspark.so`` (see ``include/spark.h``).
+The method is the one of the paper-notes page "Spark Transformer: Reactivating
+Sparsity in FFN and Attention", section 方法详解/关键设计 ("Spark FFN",
+"Statistical Top-k"):
+
+    x     = K1^T q[:r]
+    theta = mean(x) + std(x) * Q(1 - k/d_ff)
+    out   = V . (GELU(max(x - theta, 0)) (.) (K2^T q[r:]))
+
+All tensors are CUDA tensors; work is enqueued on the current (or given)
+stream.  Weights: K1 bf16 [d_ff, r], K2 bf16 [d_ff, d_model - r], V bf16
+[d_ff, d_model]; tokens q bf16 [d_model] or [T, d_model].
+"""
+from __future__ import annotations
+
+from . import _binding
+from ._binding import SparkError
+
+__all__ = ["ffn_forward", "ffn_forward_debug", "stat_topk_soft_threshold", "query_status", "release_workspace",
+           "topk_quantile", "set_wait_limit_ns", "selftest_wait_timeout", "SparkError"]
+
+
+def _require(t, name, dtype, ndim=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() not in ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _ffn_shapes(q, K1, K2, V):
+    import torch
+    for t, n in ((q, "q"), (K1, "K1"), (K2, "K2"), (V, "V")):
+        _require(t, n, torch.bfloat16)
+    d_ff, r = K1.shape
+    T = 1 if q.dim() == 1 else q.shape[0]
+    d_model = q.shape[-1]
+    if K2.shape != (d_ff, d_model - r) or V.shape != (d_ff, d_model):
+        raise ValueError(f"inconsistent shapes: K1 {tuple(K1.shape)}, K2 {tuple(K2.shape)}, V {tuple(V.shape)}, "
+                         f"q {tuple(q.shape)}")
+    return T, d_model, r, d_ff
+
+
+def ffn_forward(q, K1, K2, V, k: int, out=None, stream=None):
+    """Spark FFN forward; returns out (bf16, same shape as q)."""
+    import torch
+    T, d_model, r, d_ff = _ffn_shapes(q, K1, K2, V)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _require(out, "out", torch.bfloat16)
+    L = _binding.lib()
+    st = _binding.stream_handle(stream)
+    if q.dim() == 1:
+        rc = L.spark_ffn_forward(q.data_ptr(), K1.data_ptr(), K2.data_ptr(), V.data_ptr(), d_model, r, d_ff, int(k),
+                                 out.data_ptr(), st)
+        _binding.check("spark_ffn_forward", rc)
+    else:
+        rc = L.spark_ffn_forward_tokens(q.data_ptr(), K1.data_ptr(), K2.data_ptr(), V.data_ptr(), T, d_model, r,
+                                        d_ff, int(k), out.data_ptr(), st)
+        _binding.check("spark_ffn_forward_tokens", rc)
+    return out
+
+
+def ffn_forward_debug(q, K1, K2, V, k: int, stream=None) -> dict:
+    """Spark FFN forward that also returns x (fp32 [T, d_ff]), theta (fp32 [T]) and the
+    active mask (uint8 [T, d_ff], 1 where x > theta) the kernels used."""
+    import torch
+    T, d_model, r, d_ff = _ffn_shapes(q, K1, K2, V)
+    q2 = q.reshape(T, d_model)
+    out = torch.empty_like(q2)
+    x = torch.empty((T, d_ff), dtype=torch.float32, device=q.device)
+    theta = torch.empty((T,), dtype=torch.float32, device=q.device)
+    active = torch.empty((T, d_ff), dtype=torch.uint8, device=q.device)
+    rc = _binding.lib().spark_ffn_forward_debug(q2.data_ptr(), K1.data_ptr(), K2.data_ptr(), V.data_ptr(), T,
+                                                d_model, r, d_ff, int(k), out.data_ptr(), x.data_ptr(),
+                                                theta.data_ptr(), active.data_ptr(), _binding.stream_handle(stream))
+    _binding.check("spark_ffn_forward_debug", rc)
+    return {"out": out.reshape(q.shape), "x": x, "theta": theta, "active": active}
+
+
+def stat_topk_soft_threshold(x, k: int, out=None, stream=None):
+    """Row-wise statistical top-k with soft threshold on fp32 [rows, d]; out may be x."""
+    import torch
+    _require(x, "x", torch.float32)
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _require(out, "out", torch.float32)
+    rc = _binding.lib().stat_topk_soft_threshold(x.data_ptr(), rows, d, int(k), out.data_ptr(),
+                                                 _binding.stream_handle(stream))
+    _binding.check("stat_topk_soft_threshold", rc)
+    return out
+
+
+def query_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status code."""
+    return int(_binding.lib().spark_query_status(_binding.stream_handle(stream)))
+
+
+def release_workspace() -> None:
+    _binding.check("spark_release_workspace", _binding.lib().spark_release_workspace())
+
+
+def topk_quantile(k: int, d: int) -> float:
+    """Q(1 - k/d) as the library computes it (host, fp64)."""
+    return float(_binding.lib().spark_topk_quantile(int(k), int(d)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _binding.check("spark_set_wait_limit_ns", _binding.lib().spark_set_wait_limit_ns(int(ns)))
+
+
+def selftest_wait_timeout(stream=None) -> int:
+    """Run the bounded-wait self-test; returns the status spark_query_status reports after it."""
+    st = _binding.stream_handle(stream)
+    _binding.check("spark_selftest_wait_timeout", _binding.lib().spark_selftest_wait_timeout(st))
+    return int(_binding.lib().spark_query_status(st))

@@ -1,0 +1,81 @@
+"""ctypes binding of libspark.so -- argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels; this module
+only checks tensor dtypes/devices/contiguity, passes raw device pointers and
+the current CUDA stream through the C ABI of ``include/spark.h``, and turns
+status codes into exceptions.  There is no fallback: if the library is
+missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libspark.so")
+
+SPARK_OK = 0
+STATUS_NAMES = {0: "SPARK_OK", -1: "SPARK_EINVAL", -2: "SPARK_EALIGN", -3: "SPARK_ECUDA", -4: "SPARK_ENOMEM",
+                -5: "SPARK_ETIMEOUT", -6: "SPARK_EDEVICE"}
+
+# Every symbol that include/spark.h declares.
+EXPORTS = ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug", "stat_topk_soft_threshold",
+           "spark_query_status", "spark_release_workspace", "spark_status_string", "spark_topk_quantile",
+           "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version")
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SparkError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libspark.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m activation_sparse_transformer_predictor_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci = ctypes.c_void_p, ctypes.c_int
+        L.spark_ffn_forward.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
+        L.spark_ffn_forward_tokens.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp]
+        L.spark_ffn_forward_debug.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
+        L.stat_topk_soft_threshold.argtypes = [vp, ci, ci, ci, vp, vp]
+        L.spark_query_status.argtypes = [vp]
+        L.spark_release_workspace.argtypes = []
+        L.spark_status_string.argtypes = [ci]
+        L.spark_status_string.restype = ctypes.c_char_p
+        L.spark_topk_quantile.argtypes = [ci, ci]
+        L.spark_topk_quantile.restype = ctypes.c_double
+        L.spark_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+        L.spark_selftest_wait_timeout.argtypes = [vp]
+        L.spark_version.argtypes = []
+        for name in ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug",
+                     "stat_topk_soft_threshold", "spark_query_status", "spark_release_workspace",
+                     "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version"):
+            getattr(L, name).restype = ci
+        _lib = L
+        return L
+
+
+def check(fn: str, status: int) -> None:
+    if status != SPARK_OK:
+        raise SparkError(fn, status)
+
+
+def ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def stream_handle(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)

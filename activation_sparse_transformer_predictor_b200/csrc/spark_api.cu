@@ -1,0 +1,319 @@
+// spark_api.cu -- the C ABI declared in include/spark.h: argument checks,
+// per-(device, stream) workspaces, the host-side quantile Q(1 - k/d), and the
+// dispatch onto the kernels.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "spark.h"
+#include "spark_device.cuh"
+#include "spark_internal.h"
+
+namespace spark {
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;  // one second
+unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool is_sm100 = false;
+  int num_sms = 0;
+  size_t smem_optin = 0;
+};
+
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+
+std::mutex g_mutex;
+std::map<int, DeviceInfo> g_devices;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_workspaces;
+
+int current_device(int* dev) {
+  return cudaGetDevice(dev) == cudaSuccess ? SPARK_OK : SPARK_ECUDA;
+}
+
+int device_info(int dev, DeviceInfo* out) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& di = g_devices[dev];
+  if (!di.probed) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return SPARK_ECUDA;
+    di.is_sm100 = prop.major == 10;
+    di.num_sms = prop.multiProcessorCount;
+    di.smem_optin = prop.sharedMemPerBlockOptin;
+    di.probed = true;
+  }
+  *out = di;
+  return di.is_sm100 ? SPARK_OK : SPARK_EDEVICE;
+}
+
+// Returns a workspace of at least `bytes` for (dev, stream).  A new or regrown
+// workspace starts with a zeroed device control block.
+int get_workspace(int dev, cudaStream_t stream, size_t bytes, void** ptr) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  Workspace& ws = g_workspaces[{dev, stream}];
+  if (ws.bytes >= bytes && ws.ptr != nullptr) {
+    *ptr = ws.ptr;
+    return SPARK_OK;
+  }
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return SPARK_ECUDA;
+  if (cap != cudaStreamCaptureStatusNone) return SPARK_ENOMEM;  // no growth inside a capture
+  if (ws.ptr != nullptr) {
+    if (cudaFreeAsync(ws.ptr, stream) != cudaSuccess) return SPARK_ECUDA;
+    ws.ptr = nullptr;
+    ws.bytes = 0;
+  }
+  size_t want = bytes < (1u << 20) ? (1u << 20) : bytes;
+  void* p = nullptr;
+  if (cudaMallocAsync(&p, want, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ENOMEM;
+  }
+  if (cudaMemsetAsync(p, 0, sizeof(DeviceControl), stream) != cudaSuccess) return SPARK_ECUDA;
+  ws.ptr = p;
+  ws.bytes = want;
+  *ptr = p;
+  return SPARK_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void* a, size_t abytes, const void* b, size_t bbytes) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bbytes && b0 < a0 + abytes;
+}
+
+// Standard-normal upper-tail quantile: z with P(Z > z) = p.  First guess from
+// the rational approximation of Abramowitz & Stegun, Handbook of Mathematical
+// Functions, eq. 26.2.23 (|error| < 4.5e-4), then Newton steps on the C
+// library's erfc: z <- z + (U(z) - p) / phi(z), U(z) = erfc(z / sqrt 2) / 2.
+double upper_tail_quantile(double p) {
+  if (!(p > 0.0) || !(p < 1.0)) return NAN;
+  const bool upper = p <= 0.5;
+  const double pp = upper ? p : 1.0 - p;
+  const double t = std::sqrt(-2.0 * std::log(pp));
+  double z = t - (2.515517 + 0.802853 * t + 0.010328 * t * t) /
+                     (1.0 + 1.432788 * t + 0.189269 * t * t + 0.001308 * t * t * t);
+  if (!upper) z = -z;
+  const double inv_sqrt2 = 0.70710678118654752440;
+  const double inv_sqrt2pi = 0.39894228040143267794;
+  for (int it = 0; it < 6; ++it) {
+    const double u = 0.5 * std::erfc(z * inv_sqrt2);
+    const double phi = inv_sqrt2pi * std::exp(-0.5 * z * z);
+    if (!(phi > 0.0)) break;
+    const double step = (u - p) / phi;
+    z += step;
+    if (std::fabs(step) < 1e-16 * (1.0 + std::fabs(z))) break;
+  }
+  return z;
+}
+
+int check_ffn_args(const void* q, const void* K1, const void* K2, const void* V, int T, int d_model, int r,
+                   int d_ff, int k, const void* out) {
+  if (!q || !K1 || !K2 || !V || !out) return SPARK_EINVAL;
+  if (T < 1 || d_model < 2 || !(r > 0 && r < d_model) || !(k > 0 && k < d_ff)) return SPARK_EINVAL;
+  if (r % 8 != 0 || d_model % 8 != 0) return SPARK_EALIGN;
+  if (!aligned16(q) || !aligned16(K1) || !aligned16(K2) || !aligned16(V) || !aligned16(out)) return SPARK_EALIGN;
+  const size_t ob = static_cast<size_t>(T) * d_model * 2;
+  if (overlaps(out, ob, q, ob) || overlaps(out, ob, K1, static_cast<size_t>(d_ff) * r * 2) ||
+      overlaps(out, ob, K2, static_cast<size_t>(d_ff) * (d_model - r) * 2) ||
+      overlaps(out, ob, V, static_cast<size_t>(d_ff) * d_model * 2))
+    return SPARK_EINVAL;
+  return SPARK_OK;
+}
+
+int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* V, int T, int d_model, int r,
+                     int d_ff, int k, void* out, float* x_out, float* theta_out, unsigned char* active_out,
+                     cudaStream_t stream, int never_arrive) {
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  const double Qd = upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff));
+  const float Q = static_cast<float>(Qd);
+
+  // The fused kernel takes up to kFusedMaxTokens tokens per launch.
+  const int group = T < kFusedMaxTokens ? T : kFusedMaxTokens;
+  const FusedPlan plan = plan_fused(group, d_model, r, d_ff, di.num_sms, di.smem_optin);
+  if (!plan.ok) return SPARK_EINVAL;  // shape not supported by this build
+  void* ws = nullptr;
+  const int wst = get_workspace(dev, stream, plan.ws_bytes, &ws);
+  if (wst != SPARK_OK) return wst;
+  const unsigned char* qb = static_cast<const unsigned char*>(q);
+  unsigned char* ob = static_cast<unsigned char*>(out);
+  for (int t0 = 0; t0 < T; t0 += group) {
+    const int g = T - t0 < group ? T - t0 : group;
+    FusedPlan pl = plan;
+    if (g != group) pl = plan_fused(g, d_model, r, d_ff, di.num_sms, di.smem_optin);
+    FusedArgs a;
+    a.q = qb + static_cast<size_t>(t0) * d_model * 2;
+    a.K1 = K1;
+    a.K2 = K2;
+    a.V = V;
+    a.out = ob + static_cast<size_t>(t0) * d_model * 2;
+    a.T = g;
+    a.d_model = d_model;
+    a.r = r;
+    a.d_ff = d_ff;
+    a.Q = Q;
+    a.x_out = x_out ? x_out + static_cast<size_t>(t0) * d_ff : nullptr;
+    a.theta_out = theta_out ? theta_out + t0 : nullptr;
+    a.active_out = active_out ? active_out + static_cast<size_t>(t0) * d_ff : nullptr;
+    a.workspace = ws;
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.never_arrive = never_arrive;
+    if (launch_fused(pl, a, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return SPARK_ECUDA;
+    }
+  }
+  return SPARK_OK;
+}
+
+}  // namespace
+}  // namespace spark
+
+using namespace spark;
+
+extern "C" {
+
+SPARK_API int spark_ffn_forward(const void* q, const void* K1, const void* K2, const void* V, int d_model, int r,
+                                int d_ff, int k, void* out, spark_stream_t stream) {
+  return spark_ffn_forward_tokens(q, K1, K2, V, 1, d_model, r, d_ff, k, out, stream);
+}
+
+SPARK_API int spark_ffn_forward_tokens(const void* q, const void* K1, const void* K2, const void* V, int n_tokens,
+                                       int d_model, int r, int d_ff, int k, void* out, spark_stream_t stream) {
+  return spark_ffn_forward_debug(q, K1, K2, V, n_tokens, d_model, r, d_ff, k, out, nullptr, nullptr, nullptr,
+                                 stream);
+}
+
+SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void* K2, const void* V, int n_tokens,
+                                      int d_model, int r, int d_ff, int k, void* out, float* x_out,
+                                      float* theta_out, unsigned char* active_out, spark_stream_t stream) {
+  if (n_tokens == 0) return SPARK_OK;
+  const int st = check_ffn_args(q, K1, K2, V, n_tokens, d_model, r, d_ff, k, out);
+  if (st != SPARK_OK) return st;
+  return ffn_forward_impl(q, K1, K2, V, n_tokens, d_model, r, d_ff, k, out, x_out, theta_out, active_out,
+                          reinterpret_cast<cudaStream_t>(stream), 0);
+}
+
+SPARK_API int stat_topk_soft_threshold(const float* x, int rows, int d, int k, float* out, spark_stream_t stream) {
+  if (rows == 0) return SPARK_OK;
+  if (!x || !out || rows < 0 || d < 2 || !(k > 0 && k < d)) return SPARK_EINVAL;
+  const size_t bytes = static_cast<size_t>(rows) * d * sizeof(float);
+  if (x != out && overlaps(x, bytes, out, bytes)) return SPARK_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 3u) return SPARK_EALIGN;
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d)));
+  if (launch_stat_topk(x, out, rows, d, Q, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return SPARK_OK;
+}
+
+SPARK_API int spark_query_status(spark_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  void* ptr = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    auto it = g_workspaces.find({dev, stream});
+    if (it == g_workspaces.end() || it->second.ptr == nullptr) return SPARK_OK;
+    ptr = it->second.ptr;
+  }
+  DeviceControl ctl;
+  if (cudaMemcpy(&ctl, ptr, sizeof ctl, cudaMemcpyDeviceToHost) != cudaSuccess) return SPARK_ECUDA;
+  if (ctl.status == kDevOk && ctl.abort == 0) return SPARK_OK;
+  if (cudaMemset(ptr, 0, sizeof ctl) != cudaSuccess) return SPARK_ECUDA;  // barrier state too
+  return ctl.status == kDevTimeout ? SPARK_ETIMEOUT : SPARK_ECUDA;
+}
+
+SPARK_API int spark_release_workspace(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int prev = 0;
+  cudaGetDevice(&prev);
+  int rc = SPARK_OK;
+  for (auto& kv : g_workspaces) {
+    if (kv.second.ptr == nullptr) continue;
+    cudaSetDevice(kv.first.first);
+    if (cudaDeviceSynchronize() != cudaSuccess || cudaFree(kv.second.ptr) != cudaSuccess) rc = SPARK_ECUDA;
+  }
+  g_workspaces.clear();
+  cudaSetDevice(prev);
+  return rc;
+}
+
+SPARK_API const char* spark_status_string(int status) {
+  switch (status) {
+    case SPARK_OK: return "SPARK_OK";
+    case SPARK_EINVAL: return "SPARK_EINVAL: invalid argument";
+    case SPARK_EALIGN: return "SPARK_EALIGN: misaligned pointer or size";
+    case SPARK_ECUDA: return "SPARK_ECUDA: CUDA error";
+    case SPARK_ENOMEM: return "SPARK_ENOMEM: workspace allocation failed";
+    case SPARK_ETIMEOUT: return "SPARK_ETIMEOUT: device wait timed out";
+    case SPARK_EDEVICE: return "SPARK_EDEVICE: device is not sm_100";
+    default: return "SPARK_UNKNOWN";
+  }
+}
+
+SPARK_API double spark_topk_quantile(int k, int d) {
+  if (!(k > 0 && k < d)) return NAN;
+  return upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d));
+}
+
+SPARK_API int spark_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
+  return SPARK_OK;
+}
+
+SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream) {
+  // A tiny valid problem whose first grid barrier waits for one arrival more
+  // than there are CTAs; every CTA records the time-out and returns.
+  const int d_model = 64, r = 32, d_ff = 256, k = 20;
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  void* buf = nullptr;
+  const size_t bytes = static_cast<size_t>(d_ff) * (r + (d_model - r) + d_model) * 2 + 2 * 2 * d_model + 1024;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMallocAsync(&buf, bytes, s) != cudaSuccess) return SPARK_ENOMEM;
+  cudaMemsetAsync(buf, 0, bytes, s);
+  unsigned char* b = static_cast<unsigned char*>(buf);
+  const void* K1 = b;
+  const void* K2 = b + static_cast<size_t>(d_ff) * r * 2;
+  const void* V = b + static_cast<size_t>(d_ff) * d_model * 2;
+  const void* q = b + static_cast<size_t>(d_ff) * 2 * d_model * 2;
+  void* out = b + static_cast<size_t>(d_ff) * 2 * d_model * 2 + 256;
+  const unsigned long long saved = g_wait_limit_ns;
+  g_wait_limit_ns = 20000000ull;  // 20 ms
+  const int rc = ffn_forward_impl(q, K1, K2, V, 1, d_model, r, d_ff, k, out, nullptr, nullptr, nullptr, s, 1);
+  g_wait_limit_ns = saved;
+  cudaFreeAsync(buf, s);
+  return rc;
+}
+
+SPARK_API int spark_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,222 @@
+// spark_device.cuh -- device-side building blocks shared by the Spark kernels:
+// bounded waits, the grid barrier, mbarrier / bulk-copy wrappers, row-statistics
+// merging and GELU.  sm_100a only.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace spark {
+
+// ----------------------------------------------------------------------------
+// Device status block.  It sits at the start of every workspace, is zeroed when
+// the workspace is allocated, and is read (and cleared) by spark_query_status.
+// ----------------------------------------------------------------------------
+enum DeviceError : unsigned { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
+
+struct DeviceControl {
+  unsigned int bar_count;  // arrivals at the current grid barrier
+  unsigned int bar_gen;    // grid-barrier generation, bumped by the last arrival
+  unsigned int status;     // first device error recorded (0 = none)
+  unsigned int abort;      // set once any CTA gave up waiting; later waits bail out
+  unsigned int where;      // which wait gave up (diagnostic)
+  unsigned int pad[11];    // keep the block 64 bytes
+};
+static_assert(sizeof(DeviceControl) == 64, "DeviceControl layout");
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void record_error(DeviceControl* ctl, unsigned code, unsigned where) {
+  if (atomicCAS(&ctl->status, 0u, code) == 0u) ctl->where = where;
+  atomicExch(&ctl->abort, 1u);
+}
+
+// Grid-wide barrier for a cooperative launch (all CTAs co-resident).  The last
+// CTA to arrive resets the arrival count and bumps the generation; the others
+// spin on the generation with a time limit.  On time-out (or when another CTA
+// already gave up) the CTA records kDevTimeout and returns false; callers then
+// skip the rest of their work.  `extra` raises the arrival target so that no
+// arrival can complete it (used only by the time-out self-test).
+__device__ __forceinline__ bool grid_barrier(DeviceControl* ctl, unsigned nblocks, unsigned extra,
+                                             uint64_t limit_ns, unsigned where, int* s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    if (ld_relaxed_gpu(&ctl->abort)) {
+      ok = 0;
+    } else {
+      const unsigned gen = ld_acquire_gpu(&ctl->bar_gen);
+      __threadfence();
+      const unsigned ticket = atomicAdd(&ctl->bar_count, 1u);
+      if (ticket == nblocks - 1u + extra) {
+        ctl->bar_count = 0u;
+        __threadfence();
+        st_release_gpu(&ctl->bar_gen, gen + 1u);
+      } else {
+        const uint64_t t0 = global_timer_ns();
+        while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
+          if (ld_relaxed_gpu(&ctl->abort)) { ok = 0; break; }
+          if (global_timer_ns() - t0 > limit_ns) {
+            record_error(ctl, kDevTimeout, where);
+            ok = 0;
+            break;
+          }
+          __nanosleep(20);
+        }
+      }
+      __threadfence();
+    }
+    *s_flag = ok;
+  }
+  __syncthreads();
+  return *s_flag != 0;
+}
+
+// ----------------------------------------------------------------------------
+// mbarrier + bulk copy (TMA engine, 1-D form) wrappers.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait on an mbarrier phase.  Returns false (and records kDevTimeout)
+// if the phase did not complete within limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, uint64_t limit_ns,
+                                                  DeviceControl* ctl, unsigned where) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > limit_ns) {
+      record_error(ctl, kDevTimeout, where);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Global -> shared bulk copy completing on an mbarrier.  dst, src 16-byte
+// aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Hint: pull [src, src+bytes) into L2.  src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// Row statistics: (count, mean, M2) partials merged with Chan et al.'s
+// pairwise update, which is exact in exact arithmetic and stable in fp32.
+// ----------------------------------------------------------------------------
+struct Moments {
+  float n, mean, m2;
+};
+
+__device__ __forceinline__ Moments merge_moments(Moments a, Moments b) {
+  const float n = a.n + b.n;
+  if (n == 0.f) return a;
+  const float delta = b.mean - a.mean;
+  const float wb = b.n / n;
+  Moments r;
+  r.n = n;
+  r.mean = a.mean + delta * wb;
+  r.m2 = a.m2 + b.m2 + delta * delta * a.n * wb;
+  return r;
+}
+
+// Fixed-shape tree over the 32 lanes (shfl_down); lane 0 holds the result.
+// Deterministic: the same inputs give the same bits on every CTA.
+__device__ __forceinline__ Moments warp_merge_moments(Moments m) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    Moments o;
+    o.n = __shfl_down_sync(0xffffffffu, m.n, off);
+    o.mean = __shfl_down_sync(0xffffffffu, m.mean, off);
+    o.m2 = __shfl_down_sync(0xffffffffu, m.m2, off);
+    m = merge_moments(m, o);
+  }
+  return m;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_down_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// GELU, tanh form: 0.5 s (1 + tanh(sqrt(2/pi) (s + 0.044715 s^3))), with the
+// CUDA math library's accurate tanhf.
+__device__ __forceinline__ float gelu_tanh(float s) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  const float inner = k0 * fmaf(0.044715f * s, s * s, s);
+  return 0.5f * s * (1.f + tanhf(inner));
+}
+
+// bf16x2 packed in a 32-bit word -> two floats (exact widening).
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  float2 r;
+  r.x = __uint_as_float(w << 16);
+  r.y = __uint_as_float(w & 0xffff0000u);
+  return r;
+}
+
+}  // namespace spark

@@ -1,0 +1,50 @@
+// spark_internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace spark {
+
+struct DeviceControl;
+
+// ---------------------------------------------------------------- stat top-k
+cudaError_t launch_stat_topk(const float* x, float* out, int rows, int d, float Q, cudaStream_t stream);
+
+// ---------------------------------------------------------------- fused decode / small-batch FFN
+constexpr int kFusedMaxTokens = 8;     // tokens per launch of the fused kernel
+constexpr int kFusedMaxChunks = 8;     // 16-byte chunks per lane: r and d_model - r <= 2048
+constexpr int kFusedMaxRowsPerCta = 256;
+
+struct FusedPlan {
+  int grid;          // CTAs (all co-resident; cooperative launch)
+  int rows_per_cta;  // neurons owned by each CTA (multiple of 8)
+  int col_width;     // output columns per CTA in the value phase (power of two, >= 8)
+  int n_col_ctas;    // CTAs that own output columns
+  size_t smem_bytes; // dynamic shared memory per CTA
+  size_t ws_bytes;   // workspace bytes (device control block included)
+  bool ok;           // false: shape does not fit the fused kernel
+};
+
+FusedPlan plan_fused(int n_tokens, int d_model, int r, int d_ff, int num_sms, size_t smem_optin);
+
+struct FusedArgs {
+  const void* q;
+  const void* K1;
+  const void* K2;
+  const void* V;
+  void* out;
+  int T, d_model, r, d_ff;
+  float Q;
+  float* x_out;
+  float* theta_out;
+  unsigned char* active_out;
+  void* workspace;           // FusedPlan::ws_bytes, device control block first
+  unsigned long long wait_limit_ns;
+  int never_arrive;          // self-test: barrier 1 can never complete
+};
+
+cudaError_t launch_fused(const FusedPlan& plan, const FusedArgs& args, cudaStream_t stream);
+
+}  // namespace spark

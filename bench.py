@@ -1,0 +1,413 @@
+"""Benchmark: Spark FFN tokens/s per layer on a Gemma-2-2B-shaped layer (B200).
+
+Headline workload: decode, T = 1 token per step, d_model 2304, r 1152, d_ff 9216,
+k 737 (8%), bf16 weights ~N(0, 1/fan_in), q ~N(0, 1) (synthetic: trained
+Gemma-2 weights are not available).  A step is one full Spark FFN layer forward
+(predictor, statistics, threshold, GELU, compaction, K2/V gather) through the
+library's C ABI.  The step cycles over 16 copies of the layer's weights
+(1.36 GB, far above the 126 MB L2), so every step reads its weights from HBM.
+
+Also reported in the same JSON line (key "also"): the batched prefill at
+T = 256 tokens, the standalone statistical top-k on 32768 x 4096 fp32 score
+rows (k = 256), both timed the same way.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this method
+has: the pages publish no code) on the host cores, on the same workload.
+
+Launch: ``python bench.py --gpus N --steps K --warmup W``; for N > 1 under
+torchrun, every rank runs an independent replica (the path has no exchange
+step) and the line reports the aggregate over ranks (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+D_MODEL, R, D_FF, K = 2304, 1152, 9216, 737
+N_COPIES = 16
+METRIC = "Spark-FFN tokens/s per layer (T=1, 256) and achieved HBM GB/s vs ~8 TB/s"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
+    ap.add_argument("--no-extra", action="store_true", help="skip the prefill / stat-topk extra lines")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def profile_traffic(name: str, sources):
+    """DRAM bytes per launch from a committed ncu summary, or None if absent or the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    for s in sources:
+        h.update(open(os.path.join(ROOT, s), "rb").read())
+    if vals.get("source_sha256") != h.hexdigest()[:16]:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def source_hash(sources):
+    h = hashlib.sha256()
+    for s in sources:
+        h.update(open(os.path.join(ROOT, s), "rb").read())
+    return h.hexdigest()[:16]
+
+
+FUSED_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/ffn_fused.cu",
+                 "activation_sparse_transformer_predictor_b200/csrc/spark_device.cuh"]
+TOPK_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/stat_topk.cu",
+                "activation_sparse_transformer_predictor_b200/csrc/spark_device.cuh"]
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier_sync(world):
+    import torch
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        torch.cuda.synchronize()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_graph(fn_list, steps, warmup, world):
+    """Capture one CUDA graph that runs every callable of fn_list once (in order), replay it so
+    that `steps` calls run in total, and return device milliseconds (CUDA events) per call."""
+    import torch
+    per_graph = len(fn_list)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        # warm up on the capture stream: the library sizes its per-stream workspace here
+        for _ in range(max(warmup, 3)):
+            for f in fn_list:
+                f()
+        s.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            for f in fn_list:
+                f()
+    torch.cuda.current_stream().wait_stream(s)
+    reps = max(1, steps // per_graph)
+    for _ in range(2):
+        g.replay()
+    barrier_sync(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(reps):
+        g.replay()
+    end.record()
+    barrier_sync(world)
+    ms = start.elapsed_time(end)
+    del g
+    return ms / (reps * per_graph), reps * per_graph
+
+
+def oracle_baseline(seconds: float, T_sample: int = 1):
+    """fp64 oracle on host cores: decode tokens/s per layer on the same synthetic layer."""
+    import numpy as np
+
+    import oracle
+    from activation_sparse_transformer_predictor_b200 import synthetic
+    w = synthetic.ffn_layer(D_MODEL, R, D_FF)
+    bits = {k: synthetic.bf16_bits(v) for k, v in w.items()}
+    cores = oracle.max_threads()
+    batch = max(1, cores)
+    done = 0
+    t0 = time.perf_counter()
+    layer_seed = 0
+    while time.perf_counter() - t0 < seconds:
+        q = synthetic.bf16_bits(synthetic.tokens(batch, D_MODEL, layer=1000 + layer_seed))
+        oracle.spark_ffn(q, bits["K1"], bits["K2"], bits["V"], R, K, n_threads=cores)
+        done += batch
+        layer_seed += 1
+    el = time.perf_counter() - t0
+    return {"value": done / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} decode tokens (batches of {batch}, one per OpenMP thread) on one "
+                      f"Gemma-shaped layer, {el:.1f} s wall"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from activation_sparse_transformer_predictor_b200 import synthetic
+    w = synthetic.ffn_layer(D_MODEL, R, D_FF)
+    bits = {k: synthetic.bf16_bits(v) for k, v in w.items()}
+    cores = oracle.max_threads()
+    q = synthetic.bf16_bits(synthetic.tokens(max(1, cores), D_MODEL))
+    for _ in range(args.warmup):
+        oracle.spark_ffn(q[:1], bits["K1"], bits["K2"], bits["V"], R, K, n_threads=1)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.spark_ffn(q[i % len(q):i % len(q) + 1], bits["K1"], bits["K2"], bits["V"], R, K, n_threads=1)
+    el = time.perf_counter() - t0
+    v = args.steps / el
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "Gemma-2-2B-shaped Spark FFN layer, decode T=1", "d_model": D_MODEL, "r": R,
+                       "d_ff": D_FF, "k": K, "tokens_per_step": 1},
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{args.steps} decode tokens, one per step, single thread"},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+
+    import activation_sparse_transformer_predictor_b200 as spark
+    from activation_sparse_transformer_predictor_b200 import _binding, synthetic
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_src = peaks()
+
+    # ---------------- inputs: one synthetic layer, cloned into N_COPIES distinct buffers
+    w = synthetic.ffn_layer(D_MODEL, R, D_FF)
+    base = {k: v.to(dev) for k, v in w.items()}
+    copies = [{k: v.clone() for k, v in base.items()} for _ in range(N_COPIES)]
+    q1 = synthetic.tokens(1, D_MODEL).to(dev)[0].contiguous()
+    out1 = torch.empty_like(q1)
+    L = _binding.lib()
+
+    # measured active count on this input (deterministic), for the algorithmic byte count
+    dbg = spark.ffn_forward_debug(q1, base["K1"], base["K2"], base["V"], K)
+    m_active = int(dbg["active"].sum().item())
+    bytes_per_token = D_FF * R * 2 + m_active * ((D_MODEL - R) + D_MODEL) * 2 + 2 * D_MODEL * 2
+
+    def decode_step(c):
+        def f():
+            st = _binding.stream_handle()
+            rc = L.spark_ffn_forward(q1.data_ptr(), c["K1"].data_ptr(), c["K2"].data_ptr(), c["V"].data_ptr(),
+                                     D_MODEL, R, D_FF, K, out1.data_ptr(), st)
+            if rc != 0:
+                raise _binding.SparkError("spark_ffn_forward", rc)
+        return f
+
+    fns = [decode_step(c) for c in copies] * 8  # 128 launches per graph
+    with ClockSampler(local) as clk:
+        ms_step, n_timed = time_graph(fns, args.steps, args.warmup, world)
+    ms_step = max_over_ranks(ms_step, world)
+    assert spark.query_status() == 0
+    tok_s = 1e3 / ms_step * world
+    achieved_gbs = bytes_per_token / (ms_step * 1e-3) / 1e9
+
+    # ---------------- end to end through the public API: pinned host q in, host out back
+    q_host = synthetic.tokens(1, D_MODEL)[0].contiguous().pin_memory()
+    out_host = torch.empty_like(q_host).pin_memory()
+    q_dev = torch.empty_like(q1)
+    e2e_steps = min(args.steps, 2000)
+    for i in range(max(args.warmup, 3)):
+        q_dev.copy_(q_host, non_blocking=True)
+        o = spark.ffn_forward(q_dev, copies[i % N_COPIES]["K1"], copies[i % N_COPIES]["K2"],
+                              copies[i % N_COPIES]["V"], K, out=out1)
+        out_host.copy_(o, non_blocking=True)
+    barrier_sync(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        c = copies[i % N_COPIES]
+        q_dev.copy_(q_host, non_blocking=True)
+        o = spark.ffn_forward(q_dev, c["K1"], c["K2"], c["V"], K, out=out1)
+        out_host.copy_(o, non_blocking=True)
+    e1.record()
+    barrier_sync(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    also = {}
+    if not args.no_extra:
+        also = extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs)
+
+    if rank == 0:
+        cpu = oracle_baseline(args.cpu_seconds) if world == 1 or rank == 0 else None
+        traffic = profile_traffic("ffn_fused_decode_gemma_T1.txt", FUSED_SOURCES)
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": n_timed,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "Gemma-2-2B-shaped Spark FFN layer, decode T=1 (one token per step)",
+                       "d_model": D_MODEL, "r": R, "d_ff": D_FF, "k": K, "tokens_per_step": 1,
+                       "active_neurons": m_active, "weights": "bf16 ~N(0,1/fan_in), q ~N(0,1), seed 1234",
+                       "l2": f"inputs larger than L2: steps cycle over {N_COPIES} weight copies "
+                             f"({N_COPIES * 2 * D_MODEL * D_FF * 2 / 1e9:.2f} GB)",
+                       "timing": "CUDA graph of 128 library calls replayed; CUDA events on the launch stream",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
+                         "frac": achieved_gbs / hbm_gbs, "traffic": traffic, "peak_source": peak_src,
+                         "frac_vs_8TBs": achieved_gbs / 8000.0, "kernel": "spark_ffn_fused_kernel<1>",
+                         "algorithmic_bytes_per_launch": bytes_per_token},
+            "cpu_baseline": cpu,
+            "e2e": {"value": 1e3 / e2e_ms * world, "unit": "tokens/s", "h2d_bytes_per_step": D_MODEL * 2,
+                    "d2h_bytes_per_step": D_MODEL * 2,
+                    "path": "public Python API per step: pinned q H2D copy, ffn_forward, out D2H copy"},
+            "gpu_launches": n_timed,
+            "clocks": clk.summary(),
+            "also": also,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
+    from activation_sparse_transformer_predictor_b200 import _binding
+    L = _binding.lib()
+    res = {}
+    # prefill T = 256
+    T = 256
+    q = synthetic.tokens(T, D_MODEL, layer=1).to(dev)
+    out = torch.empty_like(q)
+
+    def pre():
+        rc = L.spark_ffn_forward_tokens(q.data_ptr(), base["K1"].data_ptr(), base["K2"].data_ptr(),
+                                        base["V"].data_ptr(), T, D_MODEL, R, D_FF, K, out.data_ptr(),
+                                        _binding.stream_handle())
+        if rc != 0:
+            raise _binding.SparkError("spark_ffn_forward_tokens", rc)
+
+    ms, n = time_graph([pre] * 4, 40, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    pred_flops = 2.0 * T * R * D_FF
+    res["prefill_T256"] = {"tokens_per_s": T * 1e3 / ms * world, "ms_per_step": ms,
+                           "predictor_tflops_effective": pred_flops / (ms * 1e-3) / 1e12,
+                           "note": "one layer, weights L2-resident (63.7 MB)"}
+    # stat top-k on 8 x 4096 x 4096 fp32 rows, k = 256
+    rows, d, k = 8 * 4096, 4096, 256
+    xs = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+    xo = torch.empty_like(xs)
+
+    def tk():
+        rc = L.stat_topk_soft_threshold(xs.data_ptr(), rows, d, k, xo.data_ptr(), _binding.stream_handle())
+        if rc != 0:
+            raise _binding.SparkError("stat_topk_soft_threshold", rc)
+
+    ms, n = time_graph([tk] * 2, 20, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    gbs = rows * d * 8 / (ms * 1e-3) / 1e9
+    res["stat_topk_32768x4096"] = {"rows_per_s": rows * 1e3 / ms * world, "ms_per_call": ms, "achieved_GBs": gbs,
+                                   "frac_of_hbm_peak": gbs / hbm_gbs,
+                                   "traffic": profile_traffic("stat_topk_32768x4096.txt", TOPK_SOURCES),
+                                   "note": "512 MiB read + 512 MiB written per call (> L2)"}
+    return res
+
+
+if __name__ == "__main__":
+    main()

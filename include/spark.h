@@ -1,0 +1,150 @@
+/*
+ * spark.h -- C ABI of libspark.so: the Spark FFN forward pass with statistical
+ * top-k, and the standalone statistical top-k operator, on NVIDIA B200 (sm_100a).
+ *
+ * Method source: the paper-notes page "Spark Transformer: Reactivating Sparsity
+ * in FFN and Attention" (NeurIPS 2025, arXiv 2506.06644), section 方法详解 /
+ * 关键设计, items "Spark FFN" and "Statistical Top-k".  Notation follows it:
+ *
+ *   x      = K1^T q[:r]                                   (low-rank predictor)
+ *   theta  = mean(x) + std(x) * Q(1 - k/d_ff)             (Q: standard-normal quantile)
+ *   s      = max(x - theta, 0)                            (Soft-Threshold)
+ *   out    = V . (GELU(s) (.) (K2^T q[r:]))               (only neurons with x > theta)
+ *
+ * Readings fixed by this library where the page is silent: std is the
+ * population standard deviation (as in LayerNorm); GELU is the tanh form; a
+ * neuron is active iff x > theta (strict); the number of active neurons is
+ * whatever theta selects (no truncation or top-up to exactly k); a row with
+ * zero spread selects nothing.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     and must stay valid until the work enqueued on `stream` has finished.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and returns once the work is enqueued.  Argument errors
+ *     are detected on the host before anything is enqueued.
+ *   - bf16 means IEEE binary32 truncated to its top 16 bits (__nv_bfloat16).
+ *     Scores x and all accumulation are fp32; out is rounded to bf16 (RNE).
+ *   - The library keeps a lazily grown scratch workspace per (device, stream),
+ *     allocated with cudaMallocAsync on `stream`.  Growing it inside a CUDA
+ *     graph capture is refused (SPARK_ENOMEM): make one call of the largest
+ *     size first.  spark_release_workspace() frees it.
+ *   - Calls made on different streams use different workspaces and may run
+ *     concurrently.
+ *   - Errors found by a kernel (a bounded wait that ran out) are recorded in a
+ *     device status word and reported by spark_query_status(); kernels never
+ *     trap.  After such an error, later launches on that stream return without
+ *     computing until spark_query_status() has been called.
+ */
+#ifndef SPARK_H_
+#define SPARK_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SPARK_API __attribute__((visibility("default")))
+#else
+#define SPARK_API
+#endif
+
+/* Same object as cudaStream_t, declared here so that this header needs no CUDA header. */
+typedef struct CUstream_st* spark_stream_t;
+
+typedef enum {
+  SPARK_OK = 0,
+  SPARK_EINVAL = -1,   /* NULL pointer, size out of range, aliasing output, unsupported shape */
+  SPARK_EALIGN = -2,   /* pointer not 16-byte aligned, or r / d_model not a multiple of 8 */
+  SPARK_ECUDA = -3,    /* a CUDA runtime call or kernel launch failed */
+  SPARK_ENOMEM = -4,   /* workspace could not be allocated (or growth requested during capture) */
+  SPARK_ETIMEOUT = -5, /* a device-side bounded wait ran out (reported by spark_query_status) */
+  SPARK_EDEVICE = -6   /* current device is not compute capability 10.x (B200 / sm_100a) */
+} spark_status;
+
+/*
+ * Spark FFN forward for one token (decode, T = 1).
+ *   q   : bf16 [d_model]          (q[:r] feeds the predictor, q[r:] the value path)
+ *   K1  : bf16 [d_ff][r]          row i is neuron i's predictor key: x_i = <K1[i,:], q[:r]>
+ *   K2  : bf16 [d_ff][d_model-r]  row i is neuron i's compute key
+ *   V   : bf16 [d_ff][d_model]    row i is neuron i's value row
+ *   out : bf16 [d_model]          must not overlap any input
+ *   k   : target number of active neurons, 0 < k < d_ff
+ * Requires 0 < r < d_model, r % 8 == 0, d_model % 8 == 0, all pointers 16-byte aligned.
+ * Returns SPARK_OK or an error code; see "Spark FFN" in the page's 关键设计.
+ */
+SPARK_API int spark_ffn_forward(const void* q, const void* K1, const void* K2, const void* V,
+                                int d_model, int r, int d_ff, int k, void* out,
+                                spark_stream_t stream);
+
+/*
+ * Same as spark_ffn_forward over n_tokens independent tokens (batched prefill):
+ * q and out are bf16 [n_tokens][d_model]; every token gets its own threshold and
+ * active set.  n_tokens == 0 is a no-op returning SPARK_OK; n_tokens < 0 is
+ * SPARK_EINVAL.
+ */
+SPARK_API int spark_ffn_forward_tokens(const void* q, const void* K1, const void* K2,
+                                       const void* V, int n_tokens, int d_model, int r, int d_ff,
+                                       int k, void* out, spark_stream_t stream);
+
+/*
+ * spark_ffn_forward_tokens that also returns the intermediate values it used,
+ * for parity checks.  Each extra output may be NULL:
+ *   x_out      : fp32 [n_tokens][d_ff]   predictor scores x
+ *   theta_out  : fp32 [n_tokens]         thresholds theta
+ *   active_out : uint8 [n_tokens][d_ff]  1 where x > theta (the neuron was used), else 0
+ * The kernels and arithmetic are the same as spark_ffn_forward_tokens.
+ */
+SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void* K2, const void* V,
+                                      int n_tokens, int d_model, int r, int d_ff, int k, void* out,
+                                      float* x_out, float* theta_out, unsigned char* active_out,
+                                      spark_stream_t stream);
+
+/*
+ * Standalone statistical top-k with soft threshold ("Statistical Top-k"):
+ * for every row of x (fp32 [rows][d]), theta = mean + std * Q(1 - k/d) and
+ * out = max(x - theta, 0) (fp32 [rows][d]).  out may equal x (in place); any
+ * other overlap is SPARK_EINVAL.  Any d >= 2 is accepted (rows need not be
+ * 16-byte aligned; aligned rows with d % 4 == 0 take the vectorised path).
+ * Requires 0 < k < d.  rows == 0 is a no-op.
+ */
+SPARK_API int stat_topk_soft_threshold(const float* x, int rows, int d, int k, float* out,
+                                       spark_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status of the
+ * workspace used on that stream: SPARK_OK, SPARK_ETIMEOUT, or SPARK_ECUDA if
+ * the stream reported a CUDA error.
+ */
+SPARK_API int spark_query_status(spark_stream_t stream);
+
+/* Synchronises the devices involved and frees every workspace.  Not thread-safe
+ * with respect to concurrent calls of the other entry points. */
+SPARK_API int spark_release_workspace(void);
+
+/* Human-readable name of a status code (static string). */
+SPARK_API const char* spark_status_string(int status);
+
+/* Q(1 - k/d) as the library computes it on the host, in double precision
+ * (rational first guess, then Newton steps on the C library's erfc).
+ * Returns NaN unless 0 < k < d. */
+SPARK_API double spark_topk_quantile(int k, int d);
+
+/* Time limit, in nanoseconds, of every device-side wait in later launches
+ * (grid barriers, copy completions).  Default 1e9 (one second); 0 restores it. */
+SPARK_API int spark_set_wait_limit_ns(unsigned long long ns);
+
+/* Self-test of the bounded waits: launches the decode kernel's grid barrier on
+ * `stream` with an arrival target that can never be met, so that every CTA runs
+ * out its time limit and records SPARK_ETIMEOUT.  Call spark_query_status() on
+ * the same stream afterwards; it must return SPARK_ETIMEOUT and clears it. */
+SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream);
+
+/* Library version: major*10000 + minor*100 + patch. */
+SPARK_API int spark_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARK_H_ */

@@ -1,0 +1,168 @@
+"""GPU parity of the Spark FFN forward against the fp64 oracle, through the C ABI.
+
+Shapes: the tiny layer (d_model 256, r 128, d_ff 1024, k 82, T 4), the
+Gemma-2-2B-shaped layer (2304 / 1152 / 9216, k 737) at decode T = 1 and a
+prefill sweep, ragged shapes and the edge cases of the method.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import activation_sparse_transformer_predictor_b200 as spark
+from activation_sparse_transformer_predictor_b200 import _binding
+
+from .gpu_util import make_layer, widen
+from .parity import assert_outputs_close, bf16_to_f64, compare_active, x_tolerance
+
+pytestmark = pytest.mark.gpu
+
+TINY = (256, 128, 1024, 82)
+GEMMA = (2304, 1152, 9216, 737)
+
+
+def run_parity(d_model, r, d_ff, k, T, layer=0, sample_tokens=None, threads=8):
+    dev, bits = make_layer(d_model, r, d_ff, T, layer=layer)
+    res = spark.ffn_forward_debug(dev["q"], dev["K1"], dev["K2"], dev["V"], k)
+    torch.cuda.synchronize()
+    assert spark.query_status() == 0
+    toks = np.arange(T) if sample_tokens is None else np.asarray(sample_tokens)
+    q_bits = bits["q"][toks]
+    orc = oracle.spark_ffn(q_bits, bits["K1"], bits["K2"], bits["V"], r, k, n_threads=threads)
+    gx = res["x"].cpu().numpy().astype(np.float64)[toks]
+    gth = res["theta"].cpu().numpy().astype(np.float64)[toks]
+    gact = res["active"].cpu().numpy().astype(bool)[toks]
+    # predictor scores within the kernel's rigorous fp32 bound
+    tol = x_tolerance(widen(bits["K1"]), widen(q_bits[:, :r]), r)
+    assert np.all(np.abs(gx - orc["x"]) <= tol)
+    # thresholds well inside the 1e-4*std band
+    assert np.all(np.abs(gth - orc["theta"]) <= 1e-5 * orc["std"])
+    # the GPU decides x > theta in fp32 on its own x and theta: reproduce exactly
+    assert np.array_equal(gact, res["x"].cpu().numpy()[toks] > res["theta"].cpu().numpy()[toks][:, None])
+    cmp = compare_active(gact, orc["x"], orc["theta"], orc["std"])
+    assert cmp["outside_band"] == 0, cmp
+    # output on the GPU's active set
+    ref = oracle.spark_ffn(q_bits, bits["K1"], bits["K2"], bits["V"], r, k, override_active=gact,
+                           n_threads=threads)["out"]
+    out = bf16_to_f64(res["out"]).reshape(T, d_model)[toks]
+    err = assert_outputs_close(out, ref)
+    # the plain entry point gives the same bits as the debug one
+    plain = spark.ffn_forward(dev["q"] if T > 1 else dev["q"][0], dev["K1"], dev["K2"], dev["V"], k)
+    assert torch.equal(plain.reshape(T, d_model), res["out"].reshape(T, d_model))
+    return err, cmp
+
+
+def test_tiny_layer_T4():
+    run_parity(*TINY, T=4)
+
+
+@pytest.mark.parametrize("layer", [0, 1, 2, 3])
+def test_gemma_decode_T1(layer):
+    err, cmp = run_parity(*GEMMA, T=1, layer=layer)
+    # selected count within Theorem 3.1's deviation (C = 1): |m - k| <= sqrt(d ln d)
+    assert abs(int(cmp["gpu_count"][0]) - 737) <= math.sqrt(9216 * math.log(9216))
+
+
+@pytest.mark.parametrize("T", [2, 3, 8, 9, 16])
+def test_gemma_small_batches(T):
+    run_parity(*GEMMA, T=T, layer=10 + T)
+
+
+@pytest.mark.parametrize("T", [64, 256])
+def test_gemma_prefill(T):
+    run_parity(*GEMMA, T=T, layer=20 + T)
+
+
+@pytest.mark.parametrize("T", [1024, 4096])
+def test_gemma_prefill_large_sampled(T):
+    rng = np.random.default_rng(T)
+    sample = np.sort(rng.choice(T, size=24, replace=False))
+    sample[0], sample[-1] = 0, T - 1
+    run_parity(*GEMMA, T=T, layer=30 + T, sample_tokens=sample)
+
+
+@pytest.mark.parametrize("shape", [
+    (264, 136, 1001, 80, 3),    # ragged d_ff: last CTA owns one neuron
+    (64, 32, 200, 17, 2),       # tiny, few CTAs
+    (512, 256, 2048, 1, 1),     # k = 1: extreme quantile
+    (512, 256, 2048, 2047, 2),  # k = d_ff - 1
+    (4096, 2048, 7104, 568, 1), # largest r and d_model - r of the fused kernel
+    (1024, 8, 4096, 328, 5),    # r = 8
+])
+def test_ragged_and_edge_shapes(shape):
+    d_model, r, d_ff, k, T = shape
+    run_parity(d_model, r, d_ff, k, T, layer=sum(shape) % 97)
+
+
+def test_degenerate_rows_select_nothing():
+    d_model, r, d_ff, k = TINY
+    dev, _ = make_layer(d_model, r, d_ff, 3)
+    q = dev["q"].clone()
+    q[0, :r] = 0  # x = 0 everywhere
+    K1 = dev["K1"].clone()
+    res = spark.ffn_forward_debug(q, K1, dev["K2"], dev["V"], k)
+    assert int(res["active"][0].sum()) == 0 and torch.all(res["out"][0] == 0)
+    K1c = K1[:1].repeat(d_ff, 1).contiguous()  # identical predictor rows: constant x
+    res = spark.ffn_forward_debug(dev["q"], K1c, dev["K2"], dev["V"], k)
+    assert int(res["active"].sum()) == 0 and torch.all(res["out"] == 0)
+
+
+@pytest.mark.parametrize("shape,T", [(GEMMA, 1), (GEMMA, 4), (TINY, 4)])
+def test_poisoned_inactive_rows_are_never_read(shape, T):
+    """NaN in every K2 / V row outside the active set leaves out bit-identical."""
+    d_model, r, d_ff, k = shape
+    dev, _ = make_layer(d_model, r, d_ff, T, layer=5)
+    res = spark.ffn_forward_debug(dev["q"], dev["K1"], dev["K2"], dev["V"], k)
+    used = res["active"].bool().any(dim=0)
+    K2p, Vp = dev["K2"].clone(), dev["V"].clone()
+    K2p[~used] = float("nan")
+    Vp[~used] = float("nan")
+    out2 = spark.ffn_forward(dev["q"], dev["K1"], K2p, Vp, k)
+    assert torch.isfinite(out2.float()).all()
+    assert torch.equal(out2, res["out"])
+
+
+def test_deterministic_across_runs():
+    d_model, r, d_ff, k = GEMMA
+    dev, _ = make_layer(d_model, r, d_ff, 3, layer=7)
+    a = spark.ffn_forward(dev["q"], dev["K1"], dev["K2"], dev["V"], k)
+    b = spark.ffn_forward(dev["q"], dev["K1"], dev["K2"], dev["V"], k)
+    assert torch.equal(a, b)
+
+
+def test_side_stream_and_empty_batch():
+    d_model, r, d_ff, k = TINY
+    dev, _ = make_layer(d_model, r, d_ff, 2)
+    ref = spark.ffn_forward(dev["q"], dev["K1"], dev["K2"], dev["V"], k)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out = spark.ffn_forward(dev["q"], dev["K1"], dev["K2"], dev["V"], k)
+    s.synchronize()
+    assert torch.equal(out, ref)
+    assert spark.query_status(s) == 0
+    empty = torch.empty((0, d_model), dtype=torch.bfloat16, device="cuda")
+    spark.ffn_forward(empty, dev["K1"], dev["K2"], dev["V"], k)
+
+
+def test_errors_are_reported_not_launched():
+    d_model, r, d_ff, k = TINY
+    dev, _ = make_layer(d_model, r, d_ff, 1)
+    with pytest.raises(_binding.SparkError) as e:
+        spark.ffn_forward(dev["q"], dev["K1"], dev["K2"], dev["V"], d_ff)
+    assert e.value.status == -1
+    with pytest.raises(_binding.SparkError) as e:
+        spark.ffn_forward(dev["q"], dev["K1"], dev["K2"], dev["V"], k, out=dev["q"])
+    assert e.value.status == -1
+    # r beyond what this build's kernels take: refused on the host
+    big = make_layer(8192, 4096, 512, 1)[0]
+    with pytest.raises(_binding.SparkError) as e:
+        spark.ffn_forward(big["q"], big["K1"], big["K2"], big["V"], 40)
+    assert e.value.status == -1
+
+
+def test_bounded_wait_times_out_and_recovers():
+    assert spark.selftest_wait_timeout() == -5  # SPARK_ETIMEOUT, then cleared
+    assert spark.query_status() == 0
+    run_parity(*TINY, T=4)

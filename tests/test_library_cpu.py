@@ -1,0 +1,81 @@
+"""libspark.so on a machine without a GPU: it loads, exports every symbol that
+include/spark.h declares, and its host-only logic (quantile, argument checks,
+status strings) behaves.  No kernel is launched here."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+import oracle
+from activation_sparse_transformer_predictor_b200 import _binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return _binding.lib()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"SPARK_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = _declared_functions()
+    assert len(declared) >= 10
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(_binding.EXPORTS)
+
+
+def test_version_and_status_strings(L):
+    assert L.spark_version() >= 100
+    assert L.spark_status_string(0) == b"SPARK_OK"
+    assert L.spark_status_string(-5).startswith(b"SPARK_ETIMEOUT")
+    assert L.spark_status_string(123) == b"SPARK_UNKNOWN"
+
+
+@pytest.mark.parametrize("d", [8, 64, 1000, 1024, 4096, 9216])
+def test_host_quantile_matches_oracle(L, d):
+    """The library's Q (rational guess + Newton on erfc) against the oracle's bisection."""
+    for k in sorted({1, 2, 3, d // 16, d // 12, int(0.08 * d), d // 2, d - 1} - {0, d}):
+        assert abs(L.spark_topk_quantile(k, d) - oracle.topk_quantile(k, d)) <= 1e-12 * max(1, abs(
+            oracle.topk_quantile(k, d))), (d, k)
+    assert math.isnan(L.spark_topk_quantile(0, d)) and math.isnan(L.spark_topk_quantile(d, d))
+
+
+def test_argument_checks_before_any_device_work(L):
+    vp = ctypes.c_void_p
+    fake = vp(1 << 20)  # never dereferenced: every case below fails validation first
+    null = vp(0)
+    EINVAL, EALIGN = -1, -2
+    f = L.spark_ffn_forward_tokens
+    assert f(null, fake, fake, fake, 1, 64, 32, 256, 20, vp(1 << 30), null) == EINVAL  # NULL q
+    assert f(fake, fake, fake, fake, -1, 64, 32, 256, 20, vp(1 << 30), null) == EINVAL  # T < 0
+    assert f(fake, fake, fake, fake, 0, 64, 32, 256, 20, vp(1 << 30), null) == 0  # empty batch: no-op
+    assert f(fake, fake, fake, fake, 1, 64, 64, 256, 20, vp(1 << 30), null) == EINVAL  # r == d_model
+    assert f(fake, fake, fake, fake, 1, 64, 0, 256, 20, vp(1 << 30), null) == EINVAL  # r == 0
+    assert f(fake, fake, fake, fake, 1, 64, 32, 256, 0, vp(1 << 30), null) == EINVAL  # k == 0
+    assert f(fake, fake, fake, fake, 1, 64, 32, 256, 256, vp(1 << 30), null) == EINVAL  # k == d_ff
+    assert f(fake, fake, fake, fake, 1, 64, 36, 256, 20, vp(1 << 30), null) == EALIGN  # r % 8
+    assert f(fake, fake, fake, fake, 1, 68, 32, 256, 20, vp(1 << 30), null) == EALIGN  # d_model % 8
+    assert f(vp((1 << 20) + 2), fake, fake, fake, 1, 64, 32, 256, 20, vp(1 << 30), null) == EALIGN
+    # out overlapping q
+    assert f(fake, vp(1 << 24), vp(1 << 25), vp(1 << 26), 1, 64, 32, 256, 20, vp((1 << 20) + 64), null) == EINVAL
+    t = L.stat_topk_soft_threshold
+    assert t(fake, 4, 100, 0, fake, null) == EINVAL
+    assert t(fake, 4, 100, 100, fake, null) == EINVAL
+    assert t(fake, 4, 1, 1, fake, null) == EINVAL
+    assert t(null, 4, 100, 10, fake, null) == EINVAL
+    assert t(fake, 0, 100, 10, fake, null) == 0  # no rows: no-op
+    assert t(fake, 4, 100, 10, vp((1 << 20) + 16), null) == EINVAL  # partial overlap
+    assert t(vp((1 << 20) + 2), 4, 100, 10, vp(1 << 30), null) == EALIGN  # not 4-byte aligned
