@@ -19,6 +19,15 @@ namespace {
 constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;  // one second
 unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
 
+// Speculative L2 prefetch margin of the decode kernel, in units of the local
+// standard deviation below the threshold (0 disables).  SPARK_SPEC_MARGIN
+// overrides it (tuning knob).
+float spec_margin_default() {
+  const char* e = std::getenv("SPARK_SPEC_MARGIN");
+  return e ? static_cast<float>(std::atof(e)) : 0.35f;
+}
+float g_spec_margin = spec_margin_default();
+
 struct DeviceInfo {
   bool probed = false;
   bool is_sm100 = false;
@@ -141,9 +150,14 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
   const double Qd = upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff));
   const float Q = static_cast<float>(Qd);
 
-  // The fused kernel takes up to kFusedMaxTokens tokens per launch.
-  const int group = T < kFusedMaxTokens ? T : kFusedMaxTokens;
-  const FusedPlan plan = plan_fused(group, d_model, r, d_ff, di.num_sms, di.smem_optin);
+  // The fused kernel takes up to kFusedMaxTokens tokens per launch; fall back
+  // to fewer tokens per launch when shared memory does not fit more.
+  int group = T < kFusedMaxTokens ? T : kFusedMaxTokens;
+  FusedPlan plan = plan_fused(group, d_model, r, d_ff, di.num_sms, di.smem_optin);
+  while (!plan.ok && group > 1) {
+    group = (group + 1) / 2;
+    plan = plan_fused(group, d_model, r, d_ff, di.num_sms, di.smem_optin);
+  }
   if (!plan.ok) return SPARK_EINVAL;  // shape not supported by this build
   void* ws = nullptr;
   const int wst = get_workspace(dev, stream, plan.ws_bytes, &ws);
@@ -165,6 +179,7 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
     a.r = r;
     a.d_ff = d_ff;
     a.Q = Q;
+    a.spec_margin = g_spec_margin;
     a.x_out = x_out ? x_out + static_cast<size_t>(t0) * d_ff : nullptr;
     a.theta_out = theta_out ? theta_out + t0 : nullptr;
     a.active_out = active_out ? active_out + static_cast<size_t>(t0) * d_ff : nullptr;

@@ -10,20 +10,26 @@
 namespace spark {
 
 // ----------------------------------------------------------------------------
-// Device status block.  It sits at the start of every workspace, is zeroed when
-// the workspace is allocated, and is read (and cleared) by spark_query_status.
+// Device control block.  It sits at the start of every workspace, is zeroed
+// when the workspace is allocated, and is read (and cleared) by
+// spark_query_status.  The arrival counters are reset by the last CTA to leave
+// each launch, so every launch starts from zeros.
 // ----------------------------------------------------------------------------
 enum DeviceError : unsigned { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
 
 struct DeviceControl {
-  unsigned int bar_count;  // arrivals at the current grid barrier
-  unsigned int bar_gen;    // grid-barrier generation, bumped by the last arrival
-  unsigned int status;     // first device error recorded (0 = none)
-  unsigned int abort;      // set once any CTA gave up waiting; later waits bail out
-  unsigned int where;      // which wait gave up (diagnostic)
-  unsigned int pad[11];    // keep the block 64 bytes
+  unsigned int status;      // first device error recorded (0 = none)
+  unsigned int abort;       // set once any CTA gave up waiting; later launches return at once
+  unsigned int where;       // which wait gave up (diagnostic)
+  unsigned int exit_count;  // CTAs that finished the current launch
+  unsigned int arrive1;     // arrivals at the statistics exchange
+  unsigned int arrive2;     // arrivals at the partial-output exchange
+  unsigned int pad0[2];
+  unsigned long long theta_word;  // published threshold of token 0 (high word) | flag (low word)
+  float theta[8];                 // published thresholds of tokens 1..7
+  unsigned int pad1[14];
 };
-static_assert(sizeof(DeviceControl) == 64, "DeviceControl layout");
+static_assert(sizeof(DeviceControl) == 128, "DeviceControl layout");
 
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
@@ -37,8 +43,14 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 
-__device__ __forceinline__ void st_release_gpu(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 __device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
@@ -47,50 +59,45 @@ __device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
   return v;
 }
 
+__device__ __forceinline__ float ld_relaxed_gpu_f32(const float* p) {
+  float v;
+  asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Release-add: this CTA's earlier writes (ordered before by __syncthreads)
+// become visible to whoever acquires the counter value it produced.
+__device__ __forceinline__ unsigned atom_add_release_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ void record_error(DeviceControl* ctl, unsigned code, unsigned where) {
   if (atomicCAS(&ctl->status, 0u, code) == 0u) ctl->where = where;
   atomicExch(&ctl->abort, 1u);
 }
 
-// Grid-wide barrier for a cooperative launch (all CTAs co-resident).  The last
-// CTA to arrive resets the arrival count and bumps the generation; the others
-// spin on the generation with a time limit.  On time-out (or when another CTA
-// already gave up) the CTA records kDevTimeout and returns false; callers then
-// skip the rest of their work.  `extra` raises the arrival target so that no
-// arrival can complete it (used only by the time-out self-test).
-__device__ __forceinline__ bool grid_barrier(DeviceControl* ctl, unsigned nblocks, unsigned extra,
-                                             uint64_t limit_ns, unsigned where, int* s_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    if (ld_relaxed_gpu(&ctl->abort)) {
-      ok = 0;
-    } else {
-      const unsigned gen = ld_acquire_gpu(&ctl->bar_gen);
-      __threadfence();
-      const unsigned ticket = atomicAdd(&ctl->bar_count, 1u);
-      if (ticket == nblocks - 1u + extra) {
-        ctl->bar_count = 0u;
-        __threadfence();
-        st_release_gpu(&ctl->bar_gen, gen + 1u);
-      } else {
-        const uint64_t t0 = global_timer_ns();
-        while (ld_acquire_gpu(&ctl->bar_gen) == gen) {
-          if (ld_relaxed_gpu(&ctl->abort)) { ok = 0; break; }
-          if (global_timer_ns() - t0 > limit_ns) {
-            record_error(ctl, kDevTimeout, where);
-            ok = 0;
-            break;
-          }
-          __nanosleep(20);
-        }
-      }
-      __threadfence();
+// Thread 0: spin until *cnt >= target (acquire), with a time limit.  Returns
+// false after recording kDevTimeout, or at once if another CTA gave up.
+__device__ __forceinline__ bool wait_count_geq(DeviceControl* ctl, const unsigned* cnt, unsigned target,
+                                               uint64_t limit_ns, unsigned where) {
+  if (ld_acquire_gpu(cnt) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (ld_acquire_gpu(cnt) < target) {
+    if (ld_relaxed_gpu(&ctl->abort)) return false;
+    if (global_timer_ns() - t0 > limit_ns) {
+      record_error(ctl, kDevTimeout, where);
+      return false;
     }
-    *s_flag = ok;
   }
-  __syncthreads();
-  return *s_flag != 0;
+  return true;
 }
 
 // ----------------------------------------------------------------------------

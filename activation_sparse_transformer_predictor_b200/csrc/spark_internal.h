@@ -13,7 +13,7 @@ struct DeviceControl;
 cudaError_t launch_stat_topk(const float* x, float* out, int rows, int d, float Q, cudaStream_t stream);
 
 // ---------------------------------------------------------------- fused decode / small-batch FFN
-constexpr int kFusedMaxTokens = 8;     // tokens per launch of the fused kernel
+constexpr int kFusedMaxTokens = 4;     // tokens per launch of the fused kernel
 constexpr int kFusedMaxChunks = 8;     // 16-byte chunks per lane: r and d_model - r <= 2048
 constexpr int kFusedMaxRowsPerCta = 256;
 
@@ -37,6 +37,7 @@ struct FusedArgs {
   void* out;
   int T, d_model, r, d_ff;
   float Q;
+  float spec_margin;         // > 0: speculative L2 prefetch of likely-active K2/V rows
   float* x_out;
   float* theta_out;
   unsigned char* active_out;
