@@ -17,12 +17,12 @@ LIB_PATH = os.path.join(PKG, "libspark.so")
 
 SPARK_OK = 0
 STATUS_NAMES = {0: "SPARK_OK", -1: "SPARK_EINVAL", -2: "SPARK_EALIGN", -3: "SPARK_ECUDA", -4: "SPARK_ENOMEM",
-                -5: "SPARK_ETIMEOUT", -6: "SPARK_EDEVICE"}
+                -5: "SPARK_ETIMEOUT", -6: "SPARK_EDEVICE", -7: "SPARK_ESCRATCH"}
 
 # Every symbol that include/spark.h declares.
 EXPORTS = ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug", "stat_topk_soft_threshold",
            "spark_query_status", "spark_release_workspace", "spark_status_string", "spark_topk_quantile",
-           "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version")
+           "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc")
 
 _lock = threading.Lock()
 _lib = None
@@ -58,9 +58,10 @@ def lib() -> ctypes.CDLL:
         L.spark_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.spark_selftest_wait_timeout.argtypes = [vp]
         L.spark_version.argtypes = []
+        L.spark_ffn_forward_noalloc.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
         for name in ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug",
                      "stat_topk_soft_threshold", "spark_query_status", "spark_release_workspace",
-                     "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version"):
+                     "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc"):
             getattr(L, name).restype = ci
         _lib = L
         return L

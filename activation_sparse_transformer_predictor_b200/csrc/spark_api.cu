@@ -287,6 +287,7 @@ SPARK_API const char* spark_status_string(int status) {
     case SPARK_ENOMEM: return "SPARK_ENOMEM: workspace allocation failed";
     case SPARK_ETIMEOUT: return "SPARK_ETIMEOUT: device wait timed out";
     case SPARK_EDEVICE: return "SPARK_EDEVICE: device is not sm_100";
+    case SPARK_ESCRATCH: return "SPARK_ESCRATCH: problem exceeds the fixed no-allocation scratch";
     default: return "SPARK_UNKNOWN";
   }
 }

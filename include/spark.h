@@ -59,7 +59,8 @@ typedef enum {
   SPARK_ECUDA = -3,    /* a CUDA runtime call or kernel launch failed */
   SPARK_ENOMEM = -4,   /* workspace could not be allocated (or growth requested during capture) */
   SPARK_ETIMEOUT = -5, /* a device-side bounded wait ran out (reported by spark_query_status) */
-  SPARK_EDEVICE = -6   /* current device is not compute capability 10.x (B200 / sm_100a) */
+  SPARK_EDEVICE = -6,  /* current device is not compute capability 10.x (B200 / sm_100a) */
+  SPARK_ESCRATCH = -7  /* spark_ffn_forward_noalloc: problem needs more than its fixed scratch */
 } spark_status;
 
 /*
@@ -139,6 +140,44 @@ SPARK_API int spark_set_wait_limit_ns(unsigned long long ns);
  * out its time limit and records SPARK_ETIMEOUT.  Call spark_query_status() on
  * the same stream afterwards; it must return SPARK_ETIMEOUT and clears it. */
 SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream);
+
+/* Size in bytes of the fixed scratch buffer used by spark_ffn_forward_noalloc. */
+#define SPARK_NOALLOC_SCRATCH_BYTES (2u << 20)
+
+/*
+ * spark_ffn_forward_noalloc -- the paper has no counterpart to this entry point;
+ * it exists for callers that must not allocate device memory while they run:
+ * for example the execute hook of an inference-engine plugin (which must not
+ * allocate), or a runtime that plans all device memory ahead of time and
+ * treats any later allocation as a failure.
+ *
+ * It computes exactly what spark_ffn_forward computes (one token, same kernel,
+ * same arguments, same argument checks) but never calls cudaMalloc,
+ * cudaMallocAsync, cudaFree or any allocating library routine.  Its scratch
+ * (control block, per-CTA moments, per-CTA partial outputs) lives in one
+ * buffer of SPARK_NOALLOC_SCRATCH_BYTES (2 MiB) compiled into the library as a
+ * static device array; every GPU that loads the library holds those 2 MiB until
+ * the process exits.  The caller still provides q, the weights and out.
+ *
+ * Limit: the problem's scratch must fit the buffer: about
+ * 4 * d_model * (number of CTAs, at most the SM count) bytes plus a few KB
+ * (1.33 MB for the Gemma-2-2B layer d_model 2304 on 148 SMs).  A larger problem
+ * returns SPARK_ESCRATCH and enqueues nothing.
+ *
+ * Set-up: the first call on a device looks up the buffer's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.
+ *
+ * Sharing: all calls on all streams use the same buffer, which keeps the last
+ * call's contents.  Each call clears the control block with a cudaMemsetAsync
+ * on `stream` before its kernel.  Calls whose work overlaps on the GPU (on
+ * different streams, or in graphs replayed concurrently) race on the buffer and
+ * give wrong results: order them.  A device-side time-out inside this entry
+ * point is not reported by spark_query_status.
+ */
+SPARK_API int spark_ffn_forward_noalloc(const void* q, const void* K1, const void* K2, const void* V,
+                                        int d_model, int r, int d_ff, int k, void* out,
+                                        spark_stream_t stream);
 
 /* Library version: major*10000 + minor*100 + patch. */
 SPARK_API int spark_version(void);
