@@ -150,6 +150,33 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
   const double Qd = upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff));
   const float Q = static_cast<float>(Qd);
 
+  if (T >= kPrefillMinTokens && d_ff % 16 == 0) {
+    void* ws = nullptr;
+    const int wst = get_workspace(dev, stream, prefill_workspace_bytes(T, d_model, d_ff, di.num_sms), &ws);
+    if (wst != SPARK_OK) return wst;
+    PrefillArgs a;
+    a.q = q;
+    a.K1 = K1;
+    a.K2 = K2;
+    a.V = V;
+    a.out = out;
+    a.T = T;
+    a.d_model = d_model;
+    a.r = r;
+    a.d_ff = d_ff;
+    a.Q = Q;
+    a.x_out = x_out;
+    a.theta_out = theta_out;
+    a.active_out = active_out;
+    a.workspace = ws;
+    a.wait_limit_ns = g_wait_limit_ns;
+    if (launch_prefill(a, di.num_sms, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return SPARK_ECUDA;
+    }
+    return SPARK_OK;
+  }
+
   // The fused kernel takes up to kFusedMaxTokens tokens per launch; fall back
   // to fewer tokens per launch when shared memory does not fit more.
   int group = T < kFusedMaxTokens ? T : kFusedMaxTokens;

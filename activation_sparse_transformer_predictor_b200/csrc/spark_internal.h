@@ -48,4 +48,26 @@ struct FusedArgs {
 
 cudaError_t launch_fused(const FusedPlan& plan, const FusedArgs& args, cudaStream_t stream);
 
+// ---------------------------------------------------------------- batched (prefill) FFN on tcgen05
+constexpr int kPrefillMinTokens = kFusedMaxTokens + 1;  // smaller batches take the fused kernel
+
+struct PrefillArgs {
+  const void* q;
+  const void* K1;
+  const void* K2;
+  const void* V;
+  void* out;
+  int T, d_model, r, d_ff;
+  float Q;
+  float* x_out;              // optional copy of the predictor scores
+  float* theta_out;
+  unsigned char* active_out;
+  void* workspace;           // prefill_workspace_bytes(), device control block first
+  unsigned long long wait_limit_ns;
+};
+
+int prefill_splitk(int T, int d_model, int d_ff, int num_sms);
+size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms);
+cudaError_t launch_prefill(const PrefillArgs& args, int num_sms, cudaStream_t stream);
+
 }  // namespace spark

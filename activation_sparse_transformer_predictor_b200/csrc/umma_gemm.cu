@@ -1,0 +1,665 @@
+// umma_gemm.cu -- batched (prefill) Spark FFN on the 5th-generation tensor cores.
+//
+// Spark Transformer notes, 关键设计 / "Spark FFN" and "Statistical Top-k", for T
+// tokens at once:
+//   GEMM 1  X = Q1 K1^T                 (predictor; x = K1^T q[:r] per token)
+//           epilogue: X in fp32 and per-(token, 128-neuron tile) moments
+//   theta   per token: merge the tile moments, theta = mean + std Q(1 - k/d_ff)
+//   GEMM 2  A = Q2 K2^T                 (K2^T q[r:] for every neuron)
+//           epilogue: h = GELU(max(x - theta, 0)) * a on x > theta, else 0, and
+//           split h = h_hi + h_lo into two bf16 matrices (h_lo = bf16(h - h_hi))
+//   GEMM 3  out = H_hi V + H_lo V        (V read once per k-block for both halves)
+//           epilogue: bf16 out, or fp32 split-K partials reduced in fixed order.
+//
+// With independent tokens the union of the per-token active sets covers almost
+// every neuron once a 128-token tile is formed (1 - 0.92^128), so the masked
+// products run as dense tiles.  h is split in two bf16 parts because a single
+// bf16 rounding of h would add ~1.7e-3 relative error on top of the bf16 output
+// rounding and break the 2e-3 relative-L2 target.
+//
+// One kernel template serves the three GEMMs: a persistent grid (one CTA per
+// SM), warp 0 = TMA producer (128B-swizzled K-major tiles; V is read N-major),
+// warp 1 = TMEM allocator and single-thread tcgen05.mma issuer (M 128, N 128,
+// K 16 per instruction, fp32 accumulators in TMEM, two accumulators so that
+// the epilogue of one tile overlaps the main loop of the next), warps 2-5 =
+// epilogue (tcgen05.ld, 32 TMEM lanes each).  Every wait is bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "spark_device.cuh"
+#include "spark_internal.h"
+
+namespace spark {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 128;
+constexpr int BK = 64;
+constexpr int kGemmThreads = 192;
+constexpr int kEpiThreads = 128;
+constexpr int kABytes = BM * BK * 2;  // 16 KB
+constexpr int kBBytes = BN * BK * 2;  // 16 KB
+
+enum Epilogue : int { kEpiPredictor = 1, kEpiGate = 2, kEpiOut = 3 };
+
+struct GemmParams {
+  int M, N, K;
+  int tiles_m, tiles_n, split_k, kb_per_split, nkb, units;
+  float* X;               // predictor scores [M][N] (written by GEMM 1, read by GEMM 2)
+  float2* moments;        // [M][tiles_n] (mean, M2) of each 128-neuron tile
+  const float* theta;     // [M]
+  uint16_t* h_hi;         // [M][N] bf16
+  uint16_t* h_lo;         // [M][N] bf16
+  unsigned char* active;  // optional [M][N]
+  float* part;            // GEMM 3 split-K partials [split][M][N]
+  uint16_t* out;          // GEMM 3 bf16 output [M][N] when split_k == 1
+  DeviceControl* ctl;
+  unsigned long long wait_limit_ns;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+// Shared-memory matrix descriptors (tcgen05 "version 1"), 128-byte swizzle.
+// K-major: rows of 128 B (64 bf16 along K), 8-row atoms 1024 B apart.
+__device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+// N-major: 64 bf16 along N per 128-byte row, one row per K index, 8-row atoms
+// 1024 B apart along K; the two 64-wide N halves of the tile are lbo bytes apart.
+__device__ __forceinline__ uint64_t desc_nmajor_sw128(uint32_t saddr, uint32_t lbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// kind::f16 instruction descriptor: bf16 A and B, fp32 D, M = 128, N = BN.
+__host__ __device__ constexpr uint32_t make_idesc(bool b_nmajor) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_nmajor ? 1u : 0u) << 16) | (static_cast<uint32_t>(BN >> 3) << 17) |
+         (static_cast<uint32_t>(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ uint16_t f2bf(float f) {
+  const __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<const uint16_t*>(&b);
+}
+
+__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+
+__device__ __forceinline__ void decode_unit(const GemmParams& p, int unit, int& tm, int& tn, int& kb0, int& kb1) {
+  const int per_split = p.tiles_m * p.tiles_n;
+  const int split = unit / per_split;
+  const int rem = unit % per_split;
+  tn = rem / p.tiles_m;  // consecutive units share an N tile: B tile reuse in L2
+  tm = rem % p.tiles_m;
+  kb0 = split * p.kb_per_split;
+  kb1 = min(p.nkb, kb0 + p.kb_per_split);
+}
+
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
+                     const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  DeviceControl* ctl = p.ctl;
+  if (ld_relaxed_gpu(&ctl->abort)) return;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], kEpiThreads);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t ph = 0;
+    int issued = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; ok && unit < p.units; unit += gridDim.x) {
+      int tm, tn, kb0, kb1;
+      decode_unit(p, unit, tm, tn, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, p.wait_limit_ns, ctl, 100) || *abort_flag) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        unsigned char* sa = smem + stage * kStageBytes;
+        mbar_arrive_expect_tx(&full[stage], kStageBytes);
+        tma_load_2d(sa, &tmA, kb * BK, tm * BM, &full[stage]);
+        if (DUAL) tma_load_2d(sa + kABytes, &tmA2, kb * BK, tm * BM, &full[stage]);
+        unsigned char* sb = sa + kABytes * (DUAL ? 2 : 1);
+        if (B_NMAJOR) {
+          tma_load_2d(sb, &tmB, tn * BN, kb * BK, &full[stage]);
+          tma_load_2d(sb + kBBytes / 2, &tmB, tn * BN + 64, kb * BK, &full[stage]);
+        } else {
+          tma_load_2d(sb, &tmB, kb * BK, tn * BN, &full[stage]);
+        }
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    if (ok) {
+      // tail: wait until the MMA warp has released every stage, so that no
+      // commit arrives on a barrier after the CTA has exited
+      for (int i = 0; i < STAGES; ++i) {
+        if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, p.wait_limit_ns, ctl, 102)) break;
+        if (++stage == STAGES) {
+          stage = 0;
+          ph ^= 1u;
+        }
+      }
+    } else {
+      // let the copies already issued land before the CTA can exit
+      int s = stage;
+      uint32_t q = ph;
+      for (int i = 0; i < STAGES && i < issued; ++i) {
+        if (--s < 0) {
+          s = STAGES - 1;
+          q ^= 1u;
+        }
+        mbar_wait_bounded(&full[s], q, p.wait_limit_ns, ctl, 101);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = make_idesc(B_NMAJOR);
+    int stage = 0;
+    uint32_t ph = 0;
+    uint32_t uses[2] = {0u, 0u};
+    int acc = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; ok && unit < p.units; unit += gridDim.x) {
+      int tm, tn, kb0, kb1;
+      decode_unit(p, unit, tm, tn, kb0, kb1);
+      if (!mbar_wait_bounded(&tempty[acc], (uses[acc] & 1u) ^ 1u, p.wait_limit_ns, ctl, 110) || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (!mbar_wait_bounded(&full[stage], ph, p.wait_limit_ns, ctl, 111) || *abort_flag) {
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + stage * kStageBytes);
+        const uint32_t sb = sa + kABytes * (DUAL ? 2 : 1);
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t bdesc = B_NMAJOR ? desc_nmajor_sw128(sb + k * 16 * 128, kBBytes / 2)
+                                          : desc_kmajor_sw128(sb + k * 32);
+          umma_bf16(d_tmem, desc_kmajor_sw128(sa + k * 32), bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          if (DUAL) umma_bf16(d_tmem, desc_kmajor_sw128(sa + kABytes + k * 32), bdesc, idesc, 1u);
+        }
+        umma_commit(&empty[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      umma_commit(&tfull[acc]);
+      ++uses[acc];
+      acc ^= 1;
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int row = quarter * 32 + lane;
+    uint32_t uses[2] = {0u, 0u};
+    int acc = 0;
+    for (int unit = blockIdx.x; unit < p.units; unit += gridDim.x) {
+      int tm, tn, kb0, kb1;
+      decode_unit(p, unit, tm, tn, kb0, kb1);
+      if (!mbar_wait_bounded(&tfull[acc], uses[acc] & 1u, p.wait_limit_ns, ctl, 120) || *abort_flag) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int m = tm * BM + row;
+      const int n_base = tn * BN;
+      const bool row_ok = m < p.M;
+      float v[16];
+      if (EPI == kEpiPredictor) {
+        float* xrow = p.X + static_cast<size_t>(m) * p.N;
+        float sum = 0.f;
+        int cnt = 0;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          tmem_ld16(taddr + c, v);
+          const int n = n_base + c;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (n + j < p.N) {
+              sum += v[j];
+              ++cnt;
+            }
+          if (row_ok) {
+            if (n + 16 <= p.N) {
+              float4* d = reinterpret_cast<float4*>(xrow + n);
+              d[0] = make_float4(v[0], v[1], v[2], v[3]);
+              d[1] = make_float4(v[4], v[5], v[6], v[7]);
+              d[2] = make_float4(v[8], v[9], v[10], v[11]);
+              d[3] = make_float4(v[12], v[13], v[14], v[15]);
+            } else {
+              for (int j = 0; j < 16; ++j)
+                if (n + j < p.N) xrow[n + j] = v[j];
+            }
+          }
+        }
+        const float mean = cnt > 0 ? sum / static_cast<float>(cnt) : 0.f;
+        float m2 = 0.f;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          tmem_ld16(taddr + c, v);
+          const int n = n_base + c;
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (n + j < p.N) {
+              const float d = v[j] - mean;
+              m2 += d * d;
+            }
+        }
+        if (row_ok) p.moments[static_cast<size_t>(m) * p.tiles_n + tn] = make_float2(mean, m2);
+      } else if (EPI == kEpiGate) {
+        const float th = row_ok ? p.theta[m] : 0.f;
+        const float* xrow = p.X + static_cast<size_t>(m) * p.N;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          tmem_ld16(taddr + c, v);
+          const int n = n_base + c;
+          if (!row_ok) continue;
+          float x[16];
+          if (n + 16 <= p.N) {
+            const float4* s4 = reinterpret_cast<const float4*>(xrow + n);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 t = __ldcg(s4 + j);
+              x[4 * j] = t.x;
+              x[4 * j + 1] = t.y;
+              x[4 * j + 2] = t.z;
+              x[4 * j + 3] = t.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[j] = n + j < p.N ? xrow[n + j] : 0.f;
+          }
+          uint32_t hi[8], lo[8];
+          uint32_t act[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            float h2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const float s = x[j + u] - th;
+              const bool a = s > 0.f && n + j + u < p.N;
+              h2[u] = a ? gelu_tanh(s) * v[j + u] : 0.f;
+              if (a) act[(j + u) >> 2] |= 1u << (8 * ((j + u) & 3));
+            }
+            const uint16_t hb0 = f2bf(h2[0]), hb1 = f2bf(h2[1]);
+            const uint16_t lb0 = f2bf(h2[0] - bf2f(hb0)), lb1 = f2bf(h2[1] - bf2f(hb1));
+            hi[j >> 1] = static_cast<uint32_t>(hb0) | (static_cast<uint32_t>(hb1) << 16);
+            lo[j >> 1] = static_cast<uint32_t>(lb0) | (static_cast<uint32_t>(lb1) << 16);
+          }
+          const size_t off = static_cast<size_t>(m) * p.N + n;
+          if (n + 16 <= p.N) {
+            uint4* dh = reinterpret_cast<uint4*>(p.h_hi + off);
+            uint4* dl = reinterpret_cast<uint4*>(p.h_lo + off);
+            dh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            dh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            dl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            if (p.active != nullptr)
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                p.active[off + j] = static_cast<unsigned char>((act[j >> 2] >> (8 * (j & 3))) & 1u);
+          } else {
+            for (int j = 0; j < 16; ++j)
+              if (n + j < p.N) {
+                p.h_hi[off + j] = static_cast<uint16_t>(hi[j >> 1] >> (16 * (j & 1)));
+                p.h_lo[off + j] = static_cast<uint16_t>(lo[j >> 1] >> (16 * (j & 1)));
+                if (p.active != nullptr) p.active[off + j] = static_cast<unsigned char>((act[j >> 2] >> (8 * (j & 3))) & 1u);
+              }
+          }
+        }
+      } else {  // kEpiOut
+        const int split = unit / (p.tiles_m * p.tiles_n);
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          tmem_ld16(taddr + c, v);
+          const int n = n_base + c;
+          if (!row_ok) continue;
+          if (p.split_k == 1) {
+            uint16_t* orow = p.out + static_cast<size_t>(m) * p.N;
+            if (n + 16 <= p.N) {
+              uint32_t w[8];
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                w[j] = static_cast<uint32_t>(f2bf(v[2 * j])) | (static_cast<uint32_t>(f2bf(v[2 * j + 1])) << 16);
+              uint4* d = reinterpret_cast<uint4*>(orow + n);
+              d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            } else {
+              for (int j = 0; j < 16; ++j)
+                if (n + j < p.N) orow[n + j] = f2bf(v[j]);
+            }
+          } else {
+            float* prow = p.part + (static_cast<size_t>(split) * p.M + m) * p.N;
+            if (n + 16 <= p.N) {
+              float4* d = reinterpret_cast<float4*>(prow + n);
+              d[0] = make_float4(v[0], v[1], v[2], v[3]);
+              d[1] = make_float4(v[4], v[5], v[6], v[7]);
+              d[2] = make_float4(v[8], v[9], v[10], v[11]);
+              d[3] = make_float4(v[12], v[13], v[14], v[15]);
+            } else {
+              for (int j = 0; j < 16; ++j)
+                if (n + j < p.N) prow[n + j] = v[j];
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      ++uses[acc];
+      acc ^= 1;
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    if (*abort_flag && lane == 0) {
+      // wait (bounded) for every MMA issued so far before TMEM is released
+      umma_commit(&tfull[0]);
+      mbar_wait_bounded(&tfull[0], 0, p.wait_limit_ns, ctl, 130);
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * BN);
+  }
+}
+
+// theta per token from the tile moments: two passes over the partials
+// (weighted mean, then M2 = sum M2_j + n_j (mean_j - mean)^2), fixed order.
+__global__ void __launch_bounds__(128) theta_kernel(const float2* moments, int M, int N, int tiles_n, float Q,
+                                                    float* theta, float* theta_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m = blockIdx.x * 4 + warp;
+  if (m >= M) return;
+  const float2* mr = moments + static_cast<size_t>(m) * tiles_n;
+  float s = 0.f;
+  for (int j = lane; j < tiles_n; j += 32) {
+    const float nj = static_cast<float>(min(BN, N - j * BN));
+    s = fmaf(nj, mr[j].x, s);
+  }
+  s = __shfl_sync(0xffffffffu, warp_sum(s), 0);
+  const float mean = s / static_cast<float>(N);
+  float m2 = 0.f;
+  for (int j = lane; j < tiles_n; j += 32) {
+    const float nj = static_cast<float>(min(BN, N - j * BN));
+    const float d = mr[j].x - mean;
+    m2 += mr[j].y + nj * d * d;
+  }
+  m2 = warp_sum(m2);
+  if (lane == 0) {
+    const float th = fmaf(sqrtf(fmaxf(m2, 0.f) / static_cast<float>(N)), Q, mean);
+    theta[m] = th;
+    if (theta_out != nullptr) theta_out[m] = th;
+  }
+}
+
+// out = bf16(sum over splits, in split order) of the GEMM 3 partials.
+__global__ void splitk_reduce_kernel(const float* part, int splits, size_t n4, uint16_t* out) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    float4 a = __ldcs(reinterpret_cast<const float4*>(part) + i);
+    for (int s = 1; s < splits; ++s) {
+      const float4 b = __ldcs(reinterpret_cast<const float4*>(part) + s * n4 + i);
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    uint2 w;
+    w.x = static_cast<uint32_t>(f2bf(a.x)) | (static_cast<uint32_t>(f2bf(a.y)) << 16);
+    w.y = static_cast<uint32_t>(f2bf(a.z)) | (static_cast<uint32_t>(f2bf(a.w)) << 16);
+    reinterpret_cast<uint2*>(out)[i] = w;
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: `inner` contiguous elements per row, `outer` rows of
+// `row_bytes`, box (box_inner x box_outer), 128-byte swizzle, zero fill.
+bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+               uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES>
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmParams& p,
+                        int num_sms, cudaStream_t stream) {
+  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes;
+  constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256;
+  auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES>;
+  static int set_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (set_dev != dev) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    set_dev = dev;
+  }
+  const int grid = p.units < num_sms ? p.units : num_sms;
+  kern<<<grid, kGemmThreads, smem, stream>>>(a, a2, b, p);
+  return cudaGetLastError();
+}
+
+size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+
+}  // namespace
+
+size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms) {
+  const int tiles_n = (d_ff + BN - 1) / BN;
+  size_t b = sizeof(DeviceControl);
+  b = align256(b) + align256(static_cast<size_t>(T) * d_ff * 4);              // X
+  b += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));            // moments
+  b += align256(static_cast<size_t>(T) * 4);                                   // theta
+  b += 2 * align256(static_cast<size_t>(T) * d_ff * 2);                        // h_hi, h_lo
+  const int splits = prefill_splitk(T, d_model, d_ff, num_sms);
+  if (splits > 1) b += align256(static_cast<size_t>(splits) * T * d_model * 4);  // partials
+  return b;
+}
+
+int prefill_splitk(int T, int d_model, int d_ff, int num_sms) {
+  const int tiles = ((T + BM - 1) / BM) * ((d_model + BN - 1) / BN);
+  const int nkb = (d_ff + BK - 1) / BK;
+  int s = 1;
+  while (tiles * s * 2 <= num_sms && s * 2 <= nkb / 4) s *= 2;
+  return s;
+}
+
+cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t stream) {
+  const int T = a.T, d_model = a.d_model, r = a.r, d2 = a.d_model - a.r, d_ff = a.d_ff;
+  const int tiles_n = (d_ff + BN - 1) / BN;
+  unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+  size_t off = align256(sizeof(DeviceControl));
+  float* X = reinterpret_cast<float*>(ws + off);
+  off += align256(static_cast<size_t>(T) * d_ff * 4);
+  float2* moments = reinterpret_cast<float2*>(ws + off);
+  off += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));
+  float* theta = reinterpret_cast<float*>(ws + off);
+  off += align256(static_cast<size_t>(T) * 4);
+  uint16_t* h_hi = reinterpret_cast<uint16_t*>(ws + off);
+  off += align256(static_cast<size_t>(T) * d_ff * 2);
+  uint16_t* h_lo = reinterpret_cast<uint16_t*>(ws + off);
+  off += align256(static_cast<size_t>(T) * d_ff * 2);
+  const int splits = prefill_splitk(T, d_model, d_ff, num_sms);
+  float* part = splits > 1 ? reinterpret_cast<float*>(ws + off) : nullptr;
+
+  const uint16_t* q = static_cast<const uint16_t*>(a.q);
+  CUtensorMap tq1, tq2, tk1, tk2, th, tl, tv;
+  const uint64_t qrow = static_cast<uint64_t>(d_model) * 2;
+  if (!make_tmap(&tq1, q, r, T, qrow, BK, BM) || !make_tmap(&tq2, q + r, d2, T, qrow, BK, BM) ||
+      !make_tmap(&tk1, a.K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, BN) ||
+      !make_tmap(&tk2, a.K2, d2, d_ff, static_cast<uint64_t>(d2) * 2, BK, BN) ||
+      !make_tmap(&th, h_hi, d_ff, T, static_cast<uint64_t>(d_ff) * 2, BK, BM) ||
+      !make_tmap(&tl, h_lo, d_ff, T, static_cast<uint64_t>(d_ff) * 2, BK, BM) ||
+      !make_tmap(&tv, a.V, d_model, d_ff, static_cast<uint64_t>(d_model) * 2, 64, BK))
+    return cudaErrorInvalidValue;
+
+  GemmParams g{};
+  g.ctl = reinterpret_cast<DeviceControl*>(ws);
+  g.wait_limit_ns = a.wait_limit_ns;
+  g.X = X;
+  g.moments = moments;
+  g.theta = theta;
+  g.h_hi = h_hi;
+  g.h_lo = h_lo;
+  g.active = a.active_out;
+  g.part = part;
+  g.out = static_cast<uint16_t*>(a.out);
+
+  // GEMM 1: X = Q1 K1^T
+  g.M = T;
+  g.N = d_ff;
+  g.K = r;
+  g.tiles_m = (T + BM - 1) / BM;
+  g.tiles_n = tiles_n;
+  g.nkb = (r + BK - 1) / BK;
+  g.split_k = 1;
+  g.kb_per_split = g.nkb;
+  g.units = g.tiles_m * g.tiles_n;
+  cudaError_t e = launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, g, num_sms, stream);
+  if (e != cudaSuccess) return e;
+  if (a.x_out != nullptr) {  // debug copy of the scores
+    e = cudaMemcpyAsync(a.x_out, X, static_cast<size_t>(T) * d_ff * 4, cudaMemcpyDeviceToDevice, stream);
+    if (e != cudaSuccess) return e;
+  }
+  theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, tiles_n, a.Q, theta, a.theta_out);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // GEMM 2: A = Q2 K2^T, gate and split
+  g.K = d2;
+  g.nkb = (d2 + BK - 1) / BK;
+  g.kb_per_split = g.nkb;
+  e = launch_gemm<kEpiGate, false, false, 6>(tq2, tq2, tk2, g, num_sms, stream);
+  if (e != cudaSuccess) return e;
+  // GEMM 3: out = H_hi V + H_lo V
+  g.N = d_model;
+  g.K = d_ff;
+  g.tiles_n = (d_model + BN - 1) / BN;
+  g.nkb = (d_ff + BK - 1) / BK;
+  g.split_k = splits;
+  g.kb_per_split = (g.nkb + splits - 1) / splits;
+  g.units = g.tiles_m * g.tiles_n * splits;
+  e = launch_gemm<kEpiOut, true, true, 4>(th, tl, tv, g, num_sms, stream);
+  if (e != cudaSuccess) return e;
+  if (splits > 1) {
+    const size_t n4 = static_cast<size_t>(T) * d_model / 4;
+    splitk_reduce_kernel<<<num_sms * 4, 256, 0, stream>>>(part, splits, n4, static_cast<uint16_t*>(a.out));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace spark
