@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill / stat-topk extra lines")
+    ap.add_argument("--case", default=None, choices=["decode", "prefill", "topk"],
+                    help="profiling mode: run only this workload, plain launches (no graph), print per-call time")
+    ap.add_argument("--tokens", type=int, default=256, help="--case prefill: tokens per call")
     return ap.parse_args()
 
 
@@ -264,10 +267,51 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_case(args):
+    """Plain launches of one workload (for ncu captures): warmup calls, then `steps` calls."""
+    import torch
+
+    import activation_sparse_transformer_predictor_b200 as spark
+    from activation_sparse_transformer_predictor_b200 import synthetic
+    dev = torch.device("cuda", 0)
+    if args.case == "topk":
+        rows, d, k = 8 * 4096, 4096, 256
+        x = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+        out = torch.empty_like(x)
+        fn = lambda i: spark.stat_topk_soft_threshold(x, k, out=out)
+        unit = f"rows {rows} x {d}"
+    else:
+        w = synthetic.ffn_layer(D_MODEL, R, D_FF)
+        copies = [{n: t.to(dev) for n, t in w.items()}]
+        if args.case == "decode":
+            copies += [{n: t.clone() for n, t in copies[0].items()} for _ in range(N_COPIES - 1)]
+            q = synthetic.tokens(1, D_MODEL).to(dev)[0].contiguous()
+        else:
+            q = synthetic.tokens(args.tokens, D_MODEL, layer=1).to(dev)
+        out = torch.empty_like(q)
+        fn = lambda i: spark.ffn_forward(q, copies[i % len(copies)]["K1"], copies[i % len(copies)]["K2"],
+                                         copies[i % len(copies)]["V"], K, out=out)
+        unit = f"{args.case}, T={1 if args.case == 'decode' else args.tokens}"
+    for i in range(args.warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(args.steps):
+        fn(args.warmup + i)
+    e1.record()
+    e1.synchronize()
+    assert spark.query_status() == 0
+    print(f"case {unit}: {e0.elapsed_time(e1) * 1e3 / args.steps:.2f} us per call over {args.steps} calls")
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.case is not None:
+        run_case(args)
         return
     import torch
 
