@@ -116,24 +116,6 @@ struct KParams {
   int never_arrive;
 };
 
-__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
-  float2 a0 = bf16x2_to_float2(a.x), b0 = bf16x2_to_float2(b.x);
-  acc = fmaf(a0.x, b0.x, acc);
-  acc = fmaf(a0.y, b0.y, acc);
-  float2 a1 = bf16x2_to_float2(a.y), b1 = bf16x2_to_float2(b.y);
-  acc = fmaf(a1.x, b1.x, acc);
-  acc = fmaf(a1.y, b1.y, acc);
-  float2 a2 = bf16x2_to_float2(a.z), b2 = bf16x2_to_float2(b.z);
-  acc = fmaf(a2.x, b2.x, acc);
-  acc = fmaf(a2.y, b2.y, acc);
-  float2 a3 = bf16x2_to_float2(a.w), b3 = bf16x2_to_float2(b.w);
-  acc = fmaf(a3.x, b3.x, acc);
-  acc = fmaf(a3.y, b3.y, acc);
-  return acc;
-}
-
-__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
-
 __device__ __forceinline__ int rows_of_cta(int c, int rpc, int d_ff) {
   const int n0 = c * rpc;
   return max(0, min(rpc, d_ff - n0));

@@ -177,6 +177,41 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
     return SPARK_OK;
   }
 
+  if (T == 1) {
+    // SPARK_DECODE_CAP (test / tuning knob): speculative candidates per CTA.
+    const char* capenv = std::getenv("SPARK_DECODE_CAP");
+    const int cap_override = capenv ? std::atoi(capenv) : -1;
+    const DecodePlan dp = plan_decode(d_model, r, d_ff, di.num_sms, di.smem_optin, cap_override);
+    if (dp.ok) {
+      void* ws = nullptr;
+      const int wst = get_workspace(dev, stream, dp.ws_bytes, &ws);
+      if (wst != SPARK_OK) return wst;
+      FusedArgs a;
+      a.q = q;
+      a.K1 = K1;
+      a.K2 = K2;
+      a.V = V;
+      a.out = out;
+      a.T = 1;
+      a.d_model = d_model;
+      a.r = r;
+      a.d_ff = d_ff;
+      a.Q = Q;
+      a.spec_margin = 0.f;
+      a.x_out = x_out;
+      a.theta_out = theta_out;
+      a.active_out = active_out;
+      a.workspace = ws;
+      a.wait_limit_ns = g_wait_limit_ns;
+      a.never_arrive = never_arrive;
+      if (launch_decode(dp, a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return SPARK_ECUDA;
+      }
+      return SPARK_OK;
+    }
+  }
+
   // The fused kernel takes up to kFusedMaxTokens tokens per launch; fall back
   // to fewer tokens per launch when shared memory does not fit more.
   int group = T < kFusedMaxTokens ? T : kFusedMaxTokens;

@@ -24,10 +24,13 @@ struct DeviceControl {
   unsigned int exit_count;  // CTAs that finished the current launch
   unsigned int arrive1;     // arrivals at the statistics exchange
   unsigned int arrive2;     // arrivals at the partial-output exchange
-  unsigned int pad0[2];
+  unsigned int s0_arrive;   // (unused)
+  unsigned int epoch;       // single-token decode launch number on this workspace
   unsigned long long theta_word;  // published threshold of token 0 (high word) | flag (low word)
   float theta[8];                 // published thresholds of tokens 1..7
-  unsigned int pad1[14];
+  unsigned int dec_arrive[2];     // single-token decode: exchange arrivals, by epoch parity
+  unsigned int dec_s0[2];         // single-token decode: first-stage arrivals, by epoch parity
+  unsigned int pad1[10];
 };
 static_assert(sizeof(DeviceControl) == 128, "DeviceControl layout");
 
@@ -84,20 +87,29 @@ __device__ __forceinline__ void record_error(DeviceControl* ctl, unsigned code, 
   atomicExch(&ctl->abort, 1u);
 }
 
+// Release-add without a return value: the arriving thread does not wait for
+// the round trip.
+__device__ __forceinline__ void red_add_release_gpu(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // Thread 0: spin until *cnt >= target (acquire), with a time limit.  Returns
-// false after recording kDevTimeout, or at once if another CTA gave up.
+// false after recording kDevTimeout, or once another CTA gave up.  The abort
+// flag and the clock are checked every 16 polls so that each poll is one load.
 __device__ __forceinline__ bool wait_count_geq(DeviceControl* ctl, const unsigned* cnt, unsigned target,
                                                uint64_t limit_ns, unsigned where) {
   if (ld_acquire_gpu(cnt) >= target) return true;
   const uint64_t t0 = global_timer_ns();
-  while (ld_acquire_gpu(cnt) < target) {
-    if (ld_relaxed_gpu(&ctl->abort)) return false;
-    if (global_timer_ns() - t0 > limit_ns) {
-      record_error(ctl, kDevTimeout, where);
-      return false;
+  for (unsigned it = 1;; ++it) {
+    if (ld_acquire_gpu(cnt) >= target) return true;
+    if ((it & 15u) == 0u) {
+      if (ld_relaxed_gpu(&ctl->abort)) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        record_error(ctl, kDevTimeout, where);
+        return false;
+      }
     }
   }
-  return true;
 }
 
 // ----------------------------------------------------------------------------
@@ -210,12 +222,15 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// GELU, tanh form: 0.5 s (1 + tanh(sqrt(2/pi) (s + 0.044715 s^3))), with the
-// CUDA math library's accurate tanhf.
+// GELU, tanh form, for s >= 0 (the kernels only evaluate it on s = x - theta > 0):
+// 0.5 s (1 + tanh(u)) with u = sqrt(2/pi) (s + 0.044715 s^3).  Uses the identity
+// 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)); for u >= 0, exp(-2u) lies in (0, 1], so
+// the quotient is well conditioned.  The fast divide (<= 2 ulp for a divisor in
+// [1, 2]) has no slow path; relative error of the result ~1e-6.
 __device__ __forceinline__ float gelu_tanh(float s) {
   const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-  const float inner = k0 * fmaf(0.044715f * s, s * s, s);
-  return 0.5f * s * (1.f + tanhf(inner));
+  const float u = k0 * fmaf(0.044715f * s, s * s, s);
+  return __fdividef(s, 1.f + __expf(-2.f * u));
 }
 
 // bf16x2 packed in a 32-bit word -> two floats (exact widening).
@@ -224,6 +239,36 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
   r.x = __uint_as_float(w << 16);
   r.y = __uint_as_float(w & 0xffff0000u);
   return r;
+}
+
+// acc + <a, b> over 8 bf16 pairs, in a fixed order (fp32 FMA).
+__device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
+  float2 a0 = bf16x2_to_float2(a.x), b0 = bf16x2_to_float2(b.x);
+  acc = fmaf(a0.x, b0.x, acc);
+  acc = fmaf(a0.y, b0.y, acc);
+  float2 a1 = bf16x2_to_float2(a.y), b1 = bf16x2_to_float2(b.y);
+  acc = fmaf(a1.x, b1.x, acc);
+  acc = fmaf(a1.y, b1.y, acc);
+  float2 a2 = bf16x2_to_float2(a.z), b2 = bf16x2_to_float2(b.z);
+  acc = fmaf(a2.x, b2.x, acc);
+  acc = fmaf(a2.y, b2.y, acc);
+  float2 a3 = bf16x2_to_float2(a.w), b3 = bf16x2_to_float2(b.w);
+  acc = fmaf(a3.x, b3.x, acc);
+  acc = fmaf(a3.y, b3.y, acc);
+  return acc;
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+__device__ __forceinline__ uint4 ldg_nc128(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+// mbarrier: add expected transaction bytes without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
 }  // namespace spark

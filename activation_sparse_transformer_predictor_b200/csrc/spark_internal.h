@@ -48,6 +48,18 @@ struct FusedArgs {
 
 cudaError_t launch_fused(const FusedPlan& plan, const FusedArgs& args, cudaStream_t stream);
 
+// ---------------------------------------------------------------- single-token decode (one exchange)
+struct DecodePlan {
+  int grid, rows_per_cta, cap, col_width, n_col_ctas;
+  size_t smem_bytes, ws_bytes;
+  bool ok;
+};
+
+// cap_override >= 0 forces the number of speculative candidates per CTA (0 makes
+// every CTA take the recompute path; used to test it).
+DecodePlan plan_decode(int d_model, int r, int d_ff, int num_sms, size_t smem_optin, int cap_override);
+cudaError_t launch_decode(const DecodePlan& plan, const FusedArgs& args, cudaStream_t stream);
+
 // ---------------------------------------------------------------- batched (prefill) FFN on tcgen05
 constexpr int kPrefillMinTokens = kFusedMaxTokens + 1;  // smaller batches take the fused kernel
 

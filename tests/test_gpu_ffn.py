@@ -166,3 +166,21 @@ def test_bounded_wait_times_out_and_recovers():
     assert spark.selftest_wait_timeout() == -5  # SPARK_ETIMEOUT, then cleared
     assert spark.query_status() == 0
     run_parity(*TINY, T=4)
+
+
+@pytest.mark.parametrize("cap", ["0", "3"])
+def test_decode_recompute_path_is_bit_identical(cap, monkeypatch):
+    """The single-token kernel speculates on candidate neurons before theta is known; a CTA
+    whose largest non-candidate score passes theta is recomputed from K1/K2 after the
+    exchange.  Forcing few or no speculation slots must give the same bits, and parity."""
+    d_model, r, d_ff, k = GEMMA
+    dev, _ = make_layer(d_model, r, d_ff, 1, layer=9)
+    q = dev["q"][0].contiguous()
+    ref = spark.ffn_forward(q, dev["K1"], dev["K2"], dev["V"], k)
+    monkeypatch.setenv("SPARK_DECODE_CAP", cap)
+    forced = spark.ffn_forward(q, dev["K1"], dev["K2"], dev["V"], k)
+    torch.cuda.synchronize()
+    assert spark.query_status() == 0
+    assert torch.equal(forced, ref)
+    monkeypatch.setenv("SPARK_DECODE_CAP", cap)
+    run_parity(*GEMMA, T=1, layer=9)
