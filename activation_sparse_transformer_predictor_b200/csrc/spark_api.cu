@@ -280,6 +280,7 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
   if (n_tokens == 0) return SPARK_OK;
   const int st = check_ffn_args(q, K1, K2, V, n_tokens, d_model, r, d_ff, k, out);
   if (st != SPARK_OK) return st;
+  if (x_out != nullptr && !aligned16(x_out)) return SPARK_EALIGN;
   return ffn_forward_impl(q, K1, K2, V, n_tokens, d_model, r, d_ff, k, out, x_out, theta_out, active_out,
                           reinterpret_cast<cudaStream_t>(stream), 0);
 }

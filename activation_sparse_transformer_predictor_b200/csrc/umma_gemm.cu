@@ -3,9 +3,13 @@
 // Spark Transformer notes, 关键设计 / "Spark FFN" and "Statistical Top-k", for T
 // tokens at once:
 //   GEMM 1  X = Q1 K1^T                 (predictor; x = K1^T q[:r] per token)
-//           epilogue: X in fp32 and per-(token, 128-neuron tile) moments
+//           epilogue: per-(token, 128-neuron tile) moments of x (x itself is
+//           stored only for the debug entry point)
 //   theta   per token: merge the tile moments, theta = mean + std Q(1 - k/d_ff)
-//   GEMM 2  A = Q2 K2^T                 (K2^T q[r:] for every neuron)
+//   GEMM 2  X = Q1 K1^T and A = Q2 K2^T  into two TMEM accumulators in one k-loop
+//           (x is recomputed on the tensor cores with the same instruction
+//           sequence as GEMM 1, so its bits are the same, instead of a 36 KB
+//           per token round trip through HBM)
 //           epilogue: h = GELU(max(x - theta, 0)) * a on x > theta, else 0, and
 //           split h = h_hi + h_lo into two bf16 matrices (h_lo = bf16(h - h_hi))
 //   GEMM 3  out = H_hi V + H_lo V        (V read once per k-block for both halves)
@@ -45,7 +49,8 @@ enum Epilogue : int { kEpiPredictor = 1, kEpiGate = 2, kEpiOut = 3 };
 struct GemmParams {
   int M, N, K;
   int tiles_m, tiles_n, split_k, kb_per_split, nkb, units;
-  float* X;               // predictor scores [M][N] (written by GEMM 1, read by GEMM 2)
+  int nkb0;               // GEMM 2: k-blocks of the first segment (Q1 K1^T); the rest is Q2 K2^T
+  float* X;               // optional predictor scores [M][N] written by GEMM 1 (debug)
   float2* moments;        // [M][tiles_n] (mean, M2) of each 128-neuron tile
   const float* theta;     // [M]
   uint16_t* h_hi;         // [M][N] bf16
@@ -146,8 +151,13 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int unit, int& 
 template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
-                     const __grid_constant__ CUtensorMap tmB, const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
+                     const GemmParams p) {
   constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes;
+  // GEMM 2 keeps two accumulators per tile (x and a): two segments of k-blocks
+  constexpr bool TWO = EPI == kEpiGate;
+  constexpr int kAccCols = TWO ? 2 * BN : BN;   // TMEM columns of one tile's accumulators
+  constexpr int kTmemCols = 2 * kAccCols;       // double buffered
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, 2 * BN);
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -196,14 +206,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         unsigned char* sa = smem + stage * kStageBytes;
         mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        tma_load_2d(sa, &tmA, kb * BK, tm * BM, &full[stage]);
-        if (DUAL) tma_load_2d(sa + kABytes, &tmA2, kb * BK, tm * BM, &full[stage]);
         unsigned char* sb = sa + kABytes * (DUAL ? 2 : 1);
-        if (B_NMAJOR) {
-          tma_load_2d(sb, &tmB, tn * BN, kb * BK, &full[stage]);
-          tma_load_2d(sb + kBBytes / 2, &tmB, tn * BN + 64, kb * BK, &full[stage]);
+        if (TWO && kb >= p.nkb0) {
+          tma_load_2d(sa, &tmA2, (kb - p.nkb0) * BK, tm * BM, &full[stage]);
+          tma_load_2d(sb, &tmB2, (kb - p.nkb0) * BK, tn * BN, &full[stage]);
         } else {
-          tma_load_2d(sb, &tmB, kb * BK, tn * BN, &full[stage]);
+          tma_load_2d(sa, &tmA, kb * BK, tm * BM, &full[stage]);
+          if (DUAL) tma_load_2d(sa + kABytes, &tmA2, kb * BK, tm * BM, &full[stage]);
+          if (B_NMAJOR) {
+            tma_load_2d(sb, &tmB, tn * BN, kb * BK, &full[stage]);
+            tma_load_2d(sb + kBBytes / 2, &tmB, tn * BN + 64, kb * BK, &full[stage]);
+          } else {
+            tma_load_2d(sb, &tmB, kb * BK, tn * BN, &full[stage]);
+          }
         }
         ++issued;
         if (++stage == STAGES) {
@@ -250,8 +265,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+      const uint32_t d_base = tmem_base + static_cast<uint32_t>(acc * kAccCols);
       for (int kb = kb0; kb < kb1; ++kb) {
+        const bool seg1 = TWO && kb >= p.nkb0;
+        const uint32_t d_tmem = d_base + (seg1 ? static_cast<uint32_t>(BN) : 0u);
+        const bool first = kb == kb0 || (TWO && kb == p.nkb0);
         if (!mbar_wait_bounded(&full[stage], ph, p.wait_limit_ns, ctl, 111) || *abort_flag) {
           *abort_flag = 1;
           ok = false;
@@ -264,7 +282,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int k = 0; k < BK / 16; ++k) {
           const uint64_t bdesc = B_NMAJOR ? desc_nmajor_sw128(sb + k * 16 * 128, kBBytes / 2)
                                           : desc_kmajor_sw128(sb + k * 32);
-          umma_bf16(d_tmem, desc_kmajor_sw128(sa + k * 32), bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          umma_bf16(d_tmem, desc_kmajor_sw128(sa + k * 32), bdesc, idesc, (!first || k > 0) ? 1u : 0u);
           if (DUAL) umma_bf16(d_tmem, desc_kmajor_sw128(sa + kABytes + k * 32), bdesc, idesc, 1u);
         }
         umma_commit(&empty[stage]);
@@ -292,7 +310,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
       const int m = tm * BM + row;
       const int n_base = tn * BN;
       const bool row_ok = m < p.M;
@@ -311,7 +329,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               sum += v[j];
               ++cnt;
             }
-          if (row_ok) {
+          if (row_ok && p.X != nullptr) {
             if (n + 16 <= p.N) {
               float4* d = reinterpret_cast<float4*>(xrow + n);
               d[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -340,27 +358,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (row_ok) p.moments[static_cast<size_t>(m) * p.tiles_n + tn] = make_float2(mean, m2);
       } else if (EPI == kEpiGate) {
         const float th = row_ok ? p.theta[m] : 0.f;
-        const float* xrow = p.X + static_cast<size_t>(m) * p.N;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
-          tmem_ld16(taddr + c, v);
+          float x[16];
+          tmem_ld16(taddr + c, x);         // recomputed scores
+          tmem_ld16(taddr + BN + c, v);    // a = K2^T q[r:]
           const int n = n_base + c;
           if (!row_ok) continue;
-          float x[16];
-          if (n + 16 <= p.N) {
-            const float4* s4 = reinterpret_cast<const float4*>(xrow + n);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float4 t = __ldcg(s4 + j);
-              x[4 * j] = t.x;
-              x[4 * j + 1] = t.y;
-              x[4 * j + 2] = t.z;
-              x[4 * j + 3] = t.w;
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) x[j] = n + j < p.N ? xrow[n + j] : 0.f;
-          }
           uint32_t hi[8], lo[8];
           uint32_t act[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
@@ -453,7 +457,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    tmem_dealloc(tmem_base, kTmemCols);
   }
 }
 
@@ -537,8 +541,8 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
 }
 
 template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES>
-cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const GemmParams& p,
-                        int num_sms, cudaStream_t stream) {
+cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const CUtensorMap& b2,
+                        const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes;
   constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256;
   auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES>;
@@ -551,7 +555,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUten
     set_dev = dev;
   }
   const int grid = p.units < num_sms ? p.units : num_sms;
-  kern<<<grid, kGemmThreads, smem, stream>>>(a, a2, b, p);
+  kern<<<grid, kGemmThreads, smem, stream>>>(a, a2, b, b2, p);
   return cudaGetLastError();
 }
 
@@ -561,8 +565,7 @@ size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms) {
   const int tiles_n = (d_ff + BN - 1) / BN;
-  size_t b = sizeof(DeviceControl);
-  b = align256(b) + align256(static_cast<size_t>(T) * d_ff * 4);              // X
+  size_t b = align256(sizeof(DeviceControl));
   b += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));            // moments
   b += align256(static_cast<size_t>(T) * 4);                                   // theta
   b += 2 * align256(static_cast<size_t>(T) * d_ff * 2);                        // h_hi, h_lo
@@ -584,8 +587,6 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   const int tiles_n = (d_ff + BN - 1) / BN;
   unsigned char* ws = static_cast<unsigned char*>(a.workspace);
   size_t off = align256(sizeof(DeviceControl));
-  float* X = reinterpret_cast<float*>(ws + off);
-  off += align256(static_cast<size_t>(T) * d_ff * 4);
   float2* moments = reinterpret_cast<float2*>(ws + off);
   off += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));
   float* theta = reinterpret_cast<float*>(ws + off);
@@ -611,7 +612,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   GemmParams g{};
   g.ctl = reinterpret_cast<DeviceControl*>(ws);
   g.wait_limit_ns = a.wait_limit_ns;
-  g.X = X;
+  g.X = a.x_out;  // scores leave the chip only for the debug entry point
   g.moments = moments;
   g.theta = theta;
   g.h_hi = h_hi;
@@ -630,19 +631,17 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   g.split_k = 1;
   g.kb_per_split = g.nkb;
   g.units = g.tiles_m * g.tiles_n;
-  cudaError_t e = launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, g, num_sms, stream);
+  cudaError_t e = launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
   if (e != cudaSuccess) return e;
-  if (a.x_out != nullptr) {  // debug copy of the scores
-    e = cudaMemcpyAsync(a.x_out, X, static_cast<size_t>(T) * d_ff * 4, cudaMemcpyDeviceToDevice, stream);
-    if (e != cudaSuccess) return e;
-  }
   theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, tiles_n, a.Q, theta, a.theta_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // GEMM 2: A = Q2 K2^T, gate and split
-  g.K = d2;
-  g.nkb = (d2 + BK - 1) / BK;
+  // GEMM 2: X = Q1 K1^T again and A = Q2 K2^T, gate and split
+  g.K = d_model;
+  g.nkb0 = (r + BK - 1) / BK;
+  g.nkb = g.nkb0 + (d2 + BK - 1) / BK;
   g.kb_per_split = g.nkb;
-  e = launch_gemm<kEpiGate, false, false, 6>(tq2, tq2, tk2, g, num_sms, stream);
+  g.X = nullptr;
+  e = launch_gemm<kEpiGate, false, false, 6>(tq1, tq2, tk1, tk2, g, num_sms, stream);
   if (e != cudaSuccess) return e;
   // GEMM 3: out = H_hi V + H_lo V
   g.N = d_model;
@@ -652,7 +651,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   g.split_k = splits;
   g.kb_per_split = (g.nkb + splits - 1) / splits;
   g.units = g.tiles_m * g.tiles_n * splits;
-  e = launch_gemm<kEpiOut, true, true, 4>(th, tl, tv, g, num_sms, stream);
+  e = launch_gemm<kEpiOut, true, true, 4>(th, tl, tv, tv, g, num_sms, stream);
   if (e != cudaSuccess) return e;
   if (splits > 1) {
     const size_t n4 = static_cast<size_t>(T) * d_model / 4;

@@ -91,7 +91,7 @@ SPARK_API int spark_ffn_forward_tokens(const void* q, const void* K1, const void
 /*
  * spark_ffn_forward_tokens that also returns the intermediate values it used,
  * for parity checks.  Each extra output may be NULL:
- *   x_out      : fp32 [n_tokens][d_ff]   predictor scores x
+ *   x_out      : fp32 [n_tokens][d_ff]   predictor scores x (16-byte aligned, else SPARK_EALIGN)
  *   theta_out  : fp32 [n_tokens]         thresholds theta
  *   active_out : uint8 [n_tokens][d_ff]  1 where x > theta (the neuron was used), else 0
  * The kernels and arithmetic are the same as spark_ffn_forward_tokens.
