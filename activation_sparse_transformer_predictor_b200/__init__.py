@@ -18,7 +18,7 @@ from __future__ import annotations
 from . import _binding
 from ._binding import SparkError
 
-__all__ = ["ffn_forward", "ffn_forward_debug", "stat_topk_soft_threshold", "query_status", "release_workspace",
+__all__ = ["ffn_forward", "ffn_forward_debug", "ffn_decode_stack", "stat_topk_soft_threshold", "query_status", "release_workspace",
            "topk_quantile", "set_wait_limit_ns", "selftest_wait_timeout", "SparkError"]
 
 
@@ -83,6 +83,33 @@ def ffn_forward_debug(q, K1, K2, V, k: int, stream=None) -> dict:
                                                 theta.data_ptr(), active.data_ptr(), _binding.stream_handle(stream))
     _binding.check("spark_ffn_forward_debug", rc)
     return {"out": out.reshape(q.shape), "x": x, "theta": theta, "active": active}
+
+
+def ffn_decode_stack(h, layers, k: int, eps: float = 1e-6, h_out=None, debug: bool = False, stream=None):
+    """Run a stack of Spark FFN layers on one token's fp32 residual h [d_model]:
+    q_l = bf16(RMSNorm(h_l)), h_{l+1} = h_l + SparkFFN_l(q_l).  `layers` is a list of
+    (K1, K2, V) bf16 CUDA tensors.  Returns h_out, or (h_out, q [L, d], out [L, d]) with debug."""
+    import ctypes
+
+    import torch
+    _require(h, "h", torch.float32, ndim=(1,))
+    d_model = h.shape[0]
+    L = len(layers)
+    for i, (K1, K2, V) in enumerate(layers):
+        _ffn_shapes(torch.empty(d_model, dtype=torch.bfloat16, device=h.device), K1, K2, V)
+    if h_out is None:
+        h_out = torch.empty_like(h)
+    d_ff, r = layers[0][0].shape if L else (1, 1)
+    ptrs = [(ctypes.c_void_p * max(L, 1))(*[t[j].data_ptr() for t in layers]) for j in range(3)]
+    qd = od = None
+    if debug:
+        qd = torch.empty((L, d_model), dtype=torch.bfloat16, device=h.device)
+        od = torch.empty((L, d_model), dtype=torch.bfloat16, device=h.device)
+    rc = _binding.lib().spark_ffn_decode_stack(h.data_ptr(), h_out.data_ptr(), ptrs[0], ptrs[1], ptrs[2], L, d_model,
+                                               r, d_ff, int(k), float(eps), _binding.ptr(qd), _binding.ptr(od),
+                                               _binding.stream_handle(stream))
+    _binding.check("spark_ffn_decode_stack", rc)
+    return (h_out, qd, od) if debug else h_out
 
 
 def stat_topk_soft_threshold(x, k: int, out=None, stream=None):

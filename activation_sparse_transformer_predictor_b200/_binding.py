@@ -22,7 +22,8 @@ STATUS_NAMES = {0: "SPARK_OK", -1: "SPARK_EINVAL", -2: "SPARK_EALIGN", -3: "SPAR
 # Every symbol that include/spark.h declares.
 EXPORTS = ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug", "stat_topk_soft_threshold",
            "spark_query_status", "spark_release_workspace", "spark_status_string", "spark_topk_quantile",
-           "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc")
+           "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc",
+           "spark_ffn_decode_stack")
 
 _lock = threading.Lock()
 _lib = None
@@ -59,9 +60,11 @@ def lib() -> ctypes.CDLL:
         L.spark_selftest_wait_timeout.argtypes = [vp]
         L.spark_version.argtypes = []
         L.spark_ffn_forward_noalloc.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
+        L.spark_ffn_decode_stack.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ctypes.c_float, vp, vp, vp]
         for name in ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug",
                      "stat_topk_soft_threshold", "spark_query_status", "spark_release_workspace",
-                     "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc"):
+                     "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc",
+           "spark_ffn_decode_stack"):
             getattr(L, name).restype = ci
         _lib = L
         return L

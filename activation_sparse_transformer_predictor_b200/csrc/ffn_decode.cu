@@ -101,6 +101,13 @@ struct DParams {
   float* x_out;
   float* theta_out;
   unsigned char* active_out;
+  // stack mode (h_in != nullptr): q = bf16(RMSNorm(h_in)) is formed in every
+  // CTA; the column owners write h_out = h_in + bf16(out) for their columns.
+  const float* h_in;
+  float* h_out;
+  float eps;
+  uint16_t* q_dbg;        // optional: the q used (bf16 [d_model]), written by CTA 0
+  const uint16_t* next_K1;  // optional: next layer's K1, prefetched into L2 after the exchange
   DeviceControl* ctl;
   float4* s0;            // [grid] (epoch tag, n, mean, M2) of each CTA's first 8 scores
   float4* hdr;           // [grid] (mean, M2, largest non-candidate x, candidate count)
@@ -170,9 +177,11 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
     mbar_init(candbar, 1);
     mbar_init(recbar, 1);
     fence_mbar_init();
-    const unsigned qbytes = static_cast<unsigned>(p.d_model) * 2;
-    mbar_arrive_expect_tx(qbar, qbytes);
-    bulk_g2s(qs, p.q, qbytes, qbar);
+    if (p.h_in == nullptr) {
+      const unsigned qbytes = static_cast<unsigned>(p.d_model) * 2;
+      mbar_arrive_expect_tx(qbar, qbytes);
+      bulk_g2s(qs, p.q, qbytes, qbar);
+    }
     for (int s = 0; s < nst; ++s) {
       const int rows = min(kRowsPerStage, nr - s * kRowsPerStage);
       const unsigned bytes = static_cast<unsigned>(rows) * p.r * 2;
@@ -186,6 +195,32 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
     misc_f[1] = -__int_as_float(0x7f800000);
   }
   __syncthreads();
+
+  if (p.h_in != nullptr) {
+    // stack mode: q = bf16(h / sqrt(mean(h^2) + eps)) while K1 streams in
+    float ss = 0.f;
+    for (int i = tid; i < p.d_model; i += kThreads) {
+      const float v = __ldcg(p.h_in + i);
+      ss = fmaf(v, v, ss);
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+      float t = 0.f;
+      for (int w = 0; w < kWarps; ++w) t += red[w];
+      misc_f[2] = 1.f / sqrtf(t / static_cast<float>(p.d_model) + p.eps);
+    }
+    __syncthreads();
+    const float inv = misc_f[2];
+    for (int i = tid; i < p.d_model; i += kThreads) {
+      const __nv_bfloat16 b = __float2bfloat16_rn(__ldcg(p.h_in + i) * inv);
+      qs[i] = *reinterpret_cast<const uint16_t*>(&b);
+      if (cta == 0 && p.q_dbg != nullptr) p.q_dbg[i] = qs[i];
+    }
+    if (tid == 0) mbar_arrive(qbar);  // q ready (no bytes in flight)
+    __syncthreads();
+  }
 
   bool ok = true;
   if (warp < kCompWarps) {
@@ -381,6 +416,15 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
   if (!misc_i[1]) return;
   if (!__syncthreads_and(mbar_wait_bounded(recbar, 0, p.wait_limit_ns, ctl, 61))) return;
 
+  // stack mode: the next layer's K1 slice goes to L2 while this layer finishes (HBM is idle now)
+  if (p.next_K1 != nullptr && tid == 0) {
+    for (int s = 0; s < nst; ++s) {
+      const int rows = min(kRowsPerStage, nr - s * kRowsPerStage);
+      prefetch_l2_bulk(p.next_K1 + static_cast<size_t>(n0 + s * kRowsPerStage) * p.r,
+                       static_cast<unsigned>(rows) * p.r * 2);
+    }
+  }
+
   // theta: every CTA merges all CTAs' moments in CTA order
   if (warp == 0) {
     float4 h[8];
@@ -538,7 +582,8 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) sum += red[(w * cpr + ch) * 8 + j];
       const __nv_bfloat16 b = __float2bfloat16_rn(sum);
-      p.out[col0 + o] = *reinterpret_cast<const uint16_t*>(&b);
+      if (p.out != nullptr) p.out[col0 + o] = *reinterpret_cast<const uint16_t*>(&b);
+      if (p.h_in != nullptr) p.h_out[col0 + o] = __ldcg(p.h_in + col0 + o) + __bfloat162float(b);
     }
   }
   // No exit bookkeeping: the next launch counts on the other parity's counters,
@@ -598,6 +643,11 @@ cudaError_t launch_decode(const DecodePlan& pl, const FusedArgs& a, cudaStream_t
   p.x_out = a.x_out;
   p.theta_out = a.theta_out;
   p.active_out = a.active_out;
+  p.h_in = a.h_in;
+  p.h_out = a.h_out;
+  p.eps = a.eps;
+  p.q_dbg = static_cast<uint16_t*>(a.q_dbg);
+  p.next_K1 = static_cast<const uint16_t*>(a.next_K1);
   p.ctl = reinterpret_cast<DeviceControl*>(ws);
   p.s0 = reinterpret_cast<float4*>(ws + W.s0);
   p.hdr = reinterpret_cast<float4*>(ws + W.hdr);

@@ -285,6 +285,74 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
                           reinterpret_cast<cudaStream_t>(stream), 0);
 }
 
+SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void* const* K1s, const void* const* K2s,
+                                     const void* const* Vs, int n_layers, int d_model, int r, int d_ff, int k,
+                                     float eps, void* q_dbg, void* out_dbg, spark_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!h_in || !h_out || n_layers < 0 || !(eps >= 0.f)) return SPARK_EINVAL;
+  if (n_layers > 0 && (!K1s || !K2s || !Vs)) return SPARK_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(h_in) | reinterpret_cast<uintptr_t>(h_out)) & 3u) return SPARK_EALIGN;
+  const size_t hb = static_cast<size_t>(d_model) * 4;
+  if (h_in != h_out && overlaps(h_in, hb, h_out, hb)) return SPARK_EINVAL;
+  if (n_layers == 0) {
+    if (h_in != h_out && cudaMemcpyAsync(h_out, h_in, hb, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
+      return SPARK_ECUDA;
+    return SPARK_OK;
+  }
+  for (int l = 0; l < n_layers; ++l) {
+    // q_l lives in the kernel's shared memory; q_dbg stands in for q in the checks
+    const int st = check_ffn_args(K1s[l], K1s[l], K2s[l], Vs[l], 1, d_model, r, d_ff, k,
+                                  out_dbg ? static_cast<unsigned char*>(out_dbg) + static_cast<size_t>(l) * d_model * 2
+                                          : reinterpret_cast<void*>(static_cast<uintptr_t>(16)));
+    if (st != SPARK_OK) return st;
+  }
+  if ((q_dbg && !aligned16(q_dbg)) || (out_dbg && !aligned16(out_dbg))) return SPARK_EALIGN;
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int dst = device_info(dev, &di);
+  if (dst != SPARK_OK) return dst;
+  const char* capenv = std::getenv("SPARK_DECODE_CAP");
+  const DecodePlan dp = plan_decode(d_model, r, d_ff, di.num_sms, di.smem_optin, capenv ? std::atoi(capenv) : -1);
+  if (!dp.ok) return SPARK_EINVAL;  // shape not supported by the single-token kernel
+  void* ws = nullptr;
+  const int wst = get_workspace(dev, stream, dp.ws_bytes, &ws);
+  if (wst != SPARK_OK) return wst;
+  const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff)));
+  for (int l = 0; l < n_layers; ++l) {
+    FusedArgs a;
+    a.q = nullptr;
+    a.K1 = K1s[l];
+    a.K2 = K2s[l];
+    a.V = Vs[l];
+    a.out = out_dbg ? static_cast<unsigned char*>(out_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
+    a.T = 1;
+    a.d_model = d_model;
+    a.r = r;
+    a.d_ff = d_ff;
+    a.Q = Q;
+    a.spec_margin = 0.f;
+    a.x_out = nullptr;
+    a.theta_out = nullptr;
+    a.active_out = nullptr;
+    a.workspace = ws;
+    a.wait_limit_ns = g_wait_limit_ns;
+    a.never_arrive = 0;
+    // every CTA reads h before it arrives at the exchange and the column owners
+    // write it after the exchange, so the update is in place from layer 1 on
+    a.h_in = l == 0 ? h_in : h_out;
+    a.h_out = h_out;
+    a.eps = eps;
+    a.q_dbg = q_dbg ? static_cast<unsigned char*>(q_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
+    a.next_K1 = l + 1 < n_layers ? K1s[l + 1] : nullptr;
+    if (launch_decode(dp, a, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return SPARK_ECUDA;
+    }
+  }
+  return SPARK_OK;
+}
+
 SPARK_API int stat_topk_soft_threshold(const float* x, int rows, int d, int k, float* out, spark_stream_t stream) {
   if (rows == 0) return SPARK_OK;
   if (!x || !out || rows < 0 || d < 2 || !(k > 0 && k < d)) return SPARK_EINVAL;

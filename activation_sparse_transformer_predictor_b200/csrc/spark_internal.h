@@ -44,6 +44,13 @@ struct FusedArgs {
   void* workspace;           // FusedPlan::ws_bytes, device control block first
   unsigned long long wait_limit_ns;
   int never_arrive;          // self-test: barrier 1 can never complete
+  // single-token stack mode (decode kernel only): q = bf16(RMSNorm(h_in)),
+  // h_out = h_in + bf16(out); nullptr h_in = plain mode
+  const float* h_in = nullptr;
+  float* h_out = nullptr;
+  float eps = 0.f;
+  void* q_dbg = nullptr;
+  const void* next_K1 = nullptr;
 };
 
 cudaError_t launch_fused(const FusedPlan& plan, const FusedArgs& args, cudaStream_t stream);

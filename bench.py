@@ -433,6 +433,34 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
     res["prefill_T256"] = {"tokens_per_s": T * 1e3 / ms * world, "ms_per_step": ms,
                            "predictor_tflops_effective": pred_flops / (ms * 1e-3) / 1e12,
                            "note": "one layer, weights L2-resident (63.7 MB)"}
+    # 26-layer decode stack (Gemma-2-2B depth), one token, residual + RMSNorm between layers
+    import ctypes
+    n_layers = 26
+    layers = []
+    for l in range(n_layers):
+        wl = synthetic.ffn_layer(D_MODEL, R, D_FF, layer=l)
+        layers.append(tuple(wl[n].to(dev) for n in ("K1", "K2", "V")))
+    ptrs = [(ctypes.c_void_p * n_layers)(*[t[j].data_ptr() for t in layers]) for j in range(3)]
+    h0 = synthetic.residual(1, D_MODEL)[0].to(dev)
+    h = h0.clone()
+
+    def stack():
+        h.copy_(h0)
+        rc = L.spark_ffn_decode_stack(h.data_ptr(), h.data_ptr(), ptrs[0], ptrs[1], ptrs[2], n_layers, D_MODEL, R,
+                                      D_FF, K, 1e-6, None, None, _binding.stream_handle())
+        if rc != 0:
+            raise _binding.SparkError("spark_ffn_decode_stack", rc)
+
+    ms, n = time_graph([stack] * 2, 20, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    stack_bytes = n_layers * (D_FF * R * 2 + 737 * (D_MODEL - R + D_MODEL) * 2 + 2 * D_MODEL * 2)
+    res["stack_26_layers_T1"] = {"tokens_per_s": 1e3 / ms * world, "us_per_token": ms * 1e3,
+                                 "us_per_layer": ms * 1e3 / n_layers,
+                                 "achieved_GBs": stack_bytes / (ms * 1e-3) / 1e9,
+                                 "frac_of_hbm_peak": stack_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
+                                 "note": "26 distinct layers (2.21 GB of weights > L2); each launch prefetches the next "
+                                         "layer's K1 into L2; bytes counted as K1 + 737 active K2/V rows + q/out per layer"}
+    del layers
     # stat top-k on 8 x 4096 x 4096 fp32 rows, k = 256
     rows, d, k = 8 * 4096, 4096, 256
     xs = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))

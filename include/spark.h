@@ -102,6 +102,25 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
                                       spark_stream_t stream);
 
 /*
+ * A decoder stack of Spark FFN layers for one token (decode).  Between layers it
+ * applies the pre-norm residual of a Gemma-style stack (the notes place Spark FFN
+ * inside a Gemma-2 model but do not spell this out; it is how the layers chain):
+ *   for l = 0 .. n_layers-1:
+ *     q_l     = bf16(h_l / sqrt(mean(h_l^2) + eps))        (RMSNorm, unit gain)
+ *     h_{l+1} = h_l + SparkFFN_l(q_l)                       (fp32 residual, bf16 FFN output)
+ *   h_in  : fp32 [d_model], h_0;  h_out : fp32 [d_model], h_{n_layers} (may equal h_in)
+ *   K1s, K2s, Vs : HOST arrays of n_layers DEVICE pointers, each as in spark_ffn_forward
+ *   q_dbg, out_dbg : optional bf16 [n_layers][d_model]: every q_l and SparkFFN_l(q_l)
+ * One launch of the single-token kernel per layer; each launch also prefetches the
+ * next layer's K1 into L2 while it finishes.  Requires the single-token kernel to
+ * support the shape (the Gemma-2-2B shape does), else SPARK_EINVAL.
+ */
+SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void* const* K1s,
+                                     const void* const* K2s, const void* const* Vs, int n_layers,
+                                     int d_model, int r, int d_ff, int k, float eps, void* q_dbg,
+                                     void* out_dbg, spark_stream_t stream);
+
+/*
  * Standalone statistical top-k with soft threshold ("Statistical Top-k"):
  * for every row of x (fp32 [rows][d]), theta = mean + std * Q(1 - k/d) and
  * out = max(x - theta, 0) (fp32 [rows][d]).  out may equal x (in place); any
