@@ -37,7 +37,8 @@ namespace spark {
 namespace {
 
 constexpr int kCompWarps = 8;
-constexpr int kWarps = kCompWarps + 1;  // + the speculation warp
+constexpr int kSpecWarp = kCompWarps;  // the speculation warp
+constexpr int kWarps = kCompWarps + 1;
 constexpr int kThreads = kWarps * 32;
 constexpr int kRowsPerStage = kCompWarps;
 constexpr int kEntryBytes = 12;  // neuron index, x, a
@@ -46,7 +47,7 @@ constexpr float kSpecSd = 6.0f;  // margin of the candidate threshold, in standa
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct DecLayout {
-  size_t region_a, cand, qs, xs, bars, cidx, red, misc, total;
+  size_t region_a, cand, qs, hsm, xs, bars, cidx, red, misc, total;
   size_t hdr_off, ent_off;  // inside region_a after phase 1
   __host__ __device__ DecLayout(int d_model, int r, int rpc, int grid, int cap) {
     const int nst = rpc / kRowsPerStage;
@@ -62,6 +63,8 @@ struct DecLayout {
     off += align_up(static_cast<size_t>(cap) * (d_model - r) * 2, 128);
     qs = off;
     off += align_up(static_cast<size_t>(d_model) * 2, 128);
+    hsm = off;  // stack mode: the fp32 residual
+    off += align_up(static_cast<size_t>(d_model) * 4, 128);
     xs = off;
     off += align_up(static_cast<size_t>(rpc) * 4, 16);
     bars = off;
@@ -107,7 +110,6 @@ struct DParams {
   float* h_out;
   float eps;
   uint16_t* q_dbg;        // optional: the q used (bf16 [d_model]), written by CTA 0
-  const uint16_t* next_K1;  // optional: next layer's K1, prefetched into L2 after the exchange
   DeviceControl* ctl;
   float4* s0;            // [grid] (epoch tag, n, mean, M2) of each CTA's first 8 scores
   float4* hdr;           // [grid] (mean, M2, largest non-candidate x, candidate count)
@@ -147,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
   uint16_t* k1s = reinterpret_cast<uint16_t*>(region_a);
   uint16_t* cand = reinterpret_cast<uint16_t*>(smem + L.cand);
   uint16_t* qs = reinterpret_cast<uint16_t*>(smem + L.qs);
+  float* hsm = reinterpret_cast<float*>(smem + L.hsm);
   float* xs = reinterpret_cast<float*>(smem + L.xs);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   int* cidx = reinterpret_cast<int*>(smem + L.cidx);
@@ -181,6 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
       const unsigned qbytes = static_cast<unsigned>(p.d_model) * 2;
       mbar_arrive_expect_tx(qbar, qbytes);
       bulk_g2s(qs, p.q, qbytes, qbar);
+    } else {
+      // stack mode: the residual first, ahead of the K1 stream
+      const unsigned hbytes = static_cast<unsigned>(p.d_model) * 4;
+      mbar_arrive_expect_tx(qbar, hbytes);
+      bulk_g2s(hsm, p.h_in, hbytes, qbar);
     }
     for (int s = 0; s < nst; ++s) {
       const int rows = min(kRowsPerStage, nr - s * kRowsPerStage);
@@ -198,9 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
 
   if (p.h_in != nullptr) {
     // stack mode: q = bf16(h / sqrt(mean(h^2) + eps)) while K1 streams in
+    const bool hok = mbar_wait_bounded(qbar, 0, p.wait_limit_ns, ctl, 8);
     float ss = 0.f;
-    for (int i = tid; i < p.d_model; i += kThreads) {
-      const float v = __ldcg(p.h_in + i);
+    for (int i = tid; hok && i < p.d_model; i += kThreads) {
+      const float v = hsm[i];
       ss = fmaf(v, v, ss);
     }
     ss = warp_sum(ss);
@@ -214,11 +223,10 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
     __syncthreads();
     const float inv = misc_f[2];
     for (int i = tid; i < p.d_model; i += kThreads) {
-      const __nv_bfloat16 b = __float2bfloat16_rn(__ldcg(p.h_in + i) * inv);
+      const __nv_bfloat16 b = __float2bfloat16_rn(hsm[i] * inv);
       qs[i] = *reinterpret_cast<const uint16_t*>(&b);
       if (cta == 0 && p.q_dbg != nullptr) p.q_dbg[i] = qs[i];
     }
-    if (tid == 0) mbar_arrive(qbar);  // q ready (no bytes in flight)
     __syncthreads();
   }
 
@@ -250,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
       __syncwarp();
       if (lane == 0) mbar_arrive(&xready[s]);
     }
-  } else {
+  } else if (warp == kSpecWarp) {
     // ------------------------------------------------------------ speculation warp
     // Launch number (its parity selects this launch's counters) and the abort
     // flag of an earlier launch that gave up waiting.
@@ -312,13 +320,15 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
     const float se = sd_e * sqrtf((1.f + 0.5f * p.Q * p.Q) / fmaxf(sn, 1.f));
     // without an estimate, speculate on nothing (the exchange then recomputes everything)
     const float cthr = (ok && sn > 1.f) ? fmaf(sd_e, p.Q, mean_e) - kSpecSd * se : __int_as_float(0x7f800000);
-    // candidates: once every stage is scored, one pass in ascending row order
-    for (int s = 0; s < nst && ok; ++s) ok = mbar_wait_bounded(&xready[s], 0, p.wait_limit_ns, ctl, 52);
+    // candidates, stage by stage as the scores land (stages already scored go
+    // at once): ascending row order, so the slots are sorted by neuron
     int ncand = 0;
     float maxnc = -__int_as_float(0x7f800000);
-    for (int base = 0; ok && base < nr; base += 32) {
-      const int li = base + lane;
-      const bool valid = li < nr;
+    for (int s = 0; ok && s < nst; ++s) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&xready[s], 0, p.wait_limit_ns, ctl, 52));
+      if (!ok) break;
+      const int li = s * kRowsPerStage + lane;
+      const bool valid = lane < kRowsPerStage && li < nr;
       const float x = valid ? xs[li] : 0.f;
       const bool c = valid && x > cthr;
       const unsigned ball = __ballot_sync(0xffffffffu, c);
@@ -415,15 +425,6 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
   __syncthreads();
   if (!misc_i[1]) return;
   if (!__syncthreads_and(mbar_wait_bounded(recbar, 0, p.wait_limit_ns, ctl, 61))) return;
-
-  // stack mode: the next layer's K1 slice goes to L2 while this layer finishes (HBM is idle now)
-  if (p.next_K1 != nullptr && tid == 0) {
-    for (int s = 0; s < nst; ++s) {
-      const int rows = min(kRowsPerStage, nr - s * kRowsPerStage);
-      prefetch_l2_bulk(p.next_K1 + static_cast<size_t>(n0 + s * kRowsPerStage) * p.r,
-                       static_cast<unsigned>(rows) * p.r * 2);
-    }
-  }
 
   // theta: every CTA merges all CTAs' moments in CTA order
   if (warp == 0) {
@@ -583,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_decode_kernel(const DPa
       for (int w = 0; w < kWarps; ++w) sum += red[(w * cpr + ch) * 8 + j];
       const __nv_bfloat16 b = __float2bfloat16_rn(sum);
       if (p.out != nullptr) p.out[col0 + o] = *reinterpret_cast<const uint16_t*>(&b);
-      if (p.h_in != nullptr) p.h_out[col0 + o] = __ldcg(p.h_in + col0 + o) + __bfloat162float(b);
+      if (p.h_in != nullptr) p.h_out[col0 + o] = hsm[col0 + o] + __bfloat162float(b);
     }
   }
   // No exit bookkeeping: the next launch counts on the other parity's counters,
@@ -647,7 +648,6 @@ cudaError_t launch_decode(const DecodePlan& pl, const FusedArgs& a, cudaStream_t
   p.h_out = a.h_out;
   p.eps = a.eps;
   p.q_dbg = static_cast<uint16_t*>(a.q_dbg);
-  p.next_K1 = static_cast<const uint16_t*>(a.next_K1);
   p.ctl = reinterpret_cast<DeviceControl*>(ws);
   p.s0 = reinterpret_cast<float4*>(ws + W.s0);
   p.hdr = reinterpret_cast<float4*>(ws + W.hdr);

@@ -291,7 +291,7 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (!h_in || !h_out || n_layers < 0 || !(eps >= 0.f)) return SPARK_EINVAL;
   if (n_layers > 0 && (!K1s || !K2s || !Vs)) return SPARK_EINVAL;
-  if ((reinterpret_cast<uintptr_t>(h_in) | reinterpret_cast<uintptr_t>(h_out)) & 3u) return SPARK_EALIGN;
+  if ((reinterpret_cast<uintptr_t>(h_in) | reinterpret_cast<uintptr_t>(h_out)) & 15u) return SPARK_EALIGN;
   const size_t hb = static_cast<size_t>(d_model) * 4;
   if (h_in != h_out && overlaps(h_in, hb, h_out, hb)) return SPARK_EINVAL;
   if (n_layers == 0) {
@@ -344,7 +344,6 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
     a.h_out = h_out;
     a.eps = eps;
     a.q_dbg = q_dbg ? static_cast<unsigned char*>(q_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
-    a.next_K1 = l + 1 < n_layers ? K1s[l + 1] : nullptr;
     if (launch_decode(dp, a, stream) != cudaSuccess) {
       cudaGetLastError();
       return SPARK_ECUDA;

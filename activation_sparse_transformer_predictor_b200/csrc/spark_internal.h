@@ -50,7 +50,6 @@ struct FusedArgs {
   float* h_out = nullptr;
   float eps = 0.f;
   void* q_dbg = nullptr;
-  const void* next_K1 = nullptr;
 };
 
 cudaError_t launch_fused(const FusedPlan& plan, const FusedArgs& args, cudaStream_t stream);

@@ -108,12 +108,13 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
  *   for l = 0 .. n_layers-1:
  *     q_l     = bf16(h_l / sqrt(mean(h_l^2) + eps))        (RMSNorm, unit gain)
  *     h_{l+1} = h_l + SparkFFN_l(q_l)                       (fp32 residual, bf16 FFN output)
- *   h_in  : fp32 [d_model], h_0;  h_out : fp32 [d_model], h_{n_layers} (may equal h_in)
+ *   h_in  : fp32 [d_model], h_0;  h_out : fp32 [d_model], h_{n_layers} (may equal h_in);
+ *           both 16-byte aligned
  *   K1s, K2s, Vs : HOST arrays of n_layers DEVICE pointers, each as in spark_ffn_forward
  *   q_dbg, out_dbg : optional bf16 [n_layers][d_model]: every q_l and SparkFFN_l(q_l)
- * One launch of the single-token kernel per layer; each launch also prefetches the
- * next layer's K1 into L2 while it finishes.  Requires the single-token kernel to
- * support the shape (the Gemma-2-2B shape does), else SPARK_EINVAL.
+ * One launch of the single-token kernel per layer; each launch forms q_l from h_l
+ * itself and writes h_{l+1}.  Requires the single-token kernel to support the
+ * shape (the Gemma-2-2B shape does), else SPARK_EINVAL.
  */
 SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void* const* K1s,
                                      const void* const* K2s, const void* const* Vs, int n_layers,
