@@ -146,6 +146,11 @@ def set_wait_limit_ns(ns: int) -> None:
     _binding.check("spark_set_wait_limit_ns", _binding.lib().spark_set_wait_limit_ns(int(ns)))
 
 
+def set_weight_overlap(enable: bool) -> None:
+    """Let the single-token score kernel stream K1 behind the preceding kernel (spark_set_weight_overlap)."""
+    _binding.check("spark_set_weight_overlap", _binding.lib().spark_set_weight_overlap(1 if enable else 0))
+
+
 def selftest_wait_timeout(stream=None) -> int:
     """Run the bounded-wait self-test; returns the status spark_query_status reports after it."""
     st = _binding.stream_handle(stream)

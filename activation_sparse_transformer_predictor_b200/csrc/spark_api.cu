@@ -28,6 +28,22 @@ float spec_margin_default() {
 }
 float g_spec_margin = spec_margin_default();
 
+// Single-token decode: whether the score kernel may stream K1 before the work
+// ahead of it on the stream has completed (spark_set_weight_overlap).
+bool g_weight_overlap = false;
+
+// Tuning / test knobs read per call: SPARK_DECODE_IMPL=exchange selects the
+// one-launch exchange kernel instead of the score + gather pair;
+// SPARK_DECODE_CLUSTER forces the gather kernel's cluster size.
+bool decode_use_exchange_kernel() {
+  const char* e = std::getenv("SPARK_DECODE_IMPL");
+  return e != nullptr && std::strcmp(e, "exchange") == 0;
+}
+int decode_cluster_override() {
+  const char* e = std::getenv("SPARK_DECODE_CLUSTER");
+  return e ? std::atoi(e) : 0;
+}
+
 struct DeviceInfo {
   bool probed = false;
   bool is_sm100 = false;
@@ -177,6 +193,36 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
     return SPARK_OK;
   }
 
+  if (T == 1 && never_arrive == 0 && !decode_use_exchange_kernel()) {
+    const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin, decode_cluster_override());
+    if (pp.ok) {
+      void* ws = nullptr;
+      const int wst = get_workspace(dev, stream, pp.ws_bytes, &ws);
+      if (wst != SPARK_OK) return wst;
+      DecodePgArgs a;
+      a.q = q;
+      a.K1 = K1;
+      a.K2 = K2;
+      a.V = V;
+      a.out = out;
+      a.d_model = d_model;
+      a.r = r;
+      a.d_ff = d_ff;
+      a.Q = Q;
+      a.x_out = x_out;
+      a.theta_out = theta_out;
+      a.active_out = active_out;
+      a.workspace = ws;
+      a.wait_limit_ns = g_wait_limit_ns;
+      a.overlap_weights = g_weight_overlap;
+      if (launch_decode_pg(pp, a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return SPARK_ECUDA;
+      }
+      return SPARK_OK;
+    }
+  }
+
   if (T == 1) {
     // SPARK_DECODE_CAP (test / tuning knob): speculative candidates per CTA.
     const char* capenv = std::getenv("SPARK_DECODE_CAP");
@@ -312,13 +358,52 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
   DeviceInfo di;
   const int dst = device_info(dev, &di);
   if (dst != SPARK_OK) return dst;
+  const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff)));
+  if (!decode_use_exchange_kernel()) {
+    const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin, decode_cluster_override());
+    if (!pp.ok) return SPARK_EINVAL;  // shape not supported by the single-token kernels
+    void* ws = nullptr;
+    const int wst = get_workspace(dev, stream, pp.ws_bytes, &ws);
+    if (wst != SPARK_OK) return wst;
+    // q_0 = bf16(RMSNorm(h_0)) into the workspace; every layer's gather kernel
+    // writes h_{l+1} and q_{l+1}
+    if (launch_rmsnorm_q(pp, ws, h_in, d_model, d_ff, eps, stream) != cudaSuccess) {
+      cudaGetLastError();
+      return SPARK_ECUDA;
+    }
+    for (int l = 0; l < n_layers; ++l) {
+      DecodePgArgs a;
+      a.K1 = K1s[l];
+      a.K2 = K2s[l];
+      a.V = Vs[l];
+      a.out = out_dbg ? static_cast<unsigned char*>(out_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
+      a.d_model = d_model;
+      a.r = r;
+      a.d_ff = d_ff;
+      a.Q = Q;
+      a.q_dbg = q_dbg ? static_cast<unsigned char*>(q_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
+      a.workspace = ws;
+      a.wait_limit_ns = g_wait_limit_ns;
+      // the kernel ahead of each score kernel is this library's own (it writes no weights)
+      a.overlap_weights = true;
+      a.q_from_workspace = true;
+      a.h_base = l == 0 ? h_in : h_out;
+      a.h_out = h_out;
+      a.write_q_next = l + 1 < n_layers;
+      a.eps = eps;
+      if (launch_decode_pg(pp, a, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return SPARK_ECUDA;
+      }
+    }
+    return SPARK_OK;
+  }
   const char* capenv = std::getenv("SPARK_DECODE_CAP");
   const DecodePlan dp = plan_decode(d_model, r, d_ff, di.num_sms, di.smem_optin, capenv ? std::atoi(capenv) : -1);
   if (!dp.ok) return SPARK_EINVAL;  // shape not supported by the single-token kernel
   void* ws = nullptr;
   const int wst = get_workspace(dev, stream, dp.ws_bytes, &ws);
   if (wst != SPARK_OK) return wst;
-  const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff)));
   for (int l = 0; l < n_layers; ++l) {
     FusedArgs a;
     a.q = nullptr;
@@ -429,6 +514,11 @@ SPARK_API double spark_topk_quantile(int k, int d) {
 
 SPARK_API int spark_set_wait_limit_ns(unsigned long long ns) {
   g_wait_limit_ns = ns == 0 ? kDefaultWaitLimitNs : ns;
+  return SPARK_OK;
+}
+
+SPARK_API int spark_set_weight_overlap(int enable) {
+  g_weight_overlap = enable != 0;
   return SPARK_OK;
 }
 

@@ -24,7 +24,7 @@ struct DeviceControl {
   unsigned int exit_count;  // CTAs that finished the current launch
   unsigned int arrive1;     // arrivals at the statistics exchange
   unsigned int arrive2;     // arrivals at the partial-output exchange
-  unsigned int s0_arrive;   // (unused)
+  unsigned int pg_arrive;   // single-token gather kernel: clusters that wrote their partial
   unsigned int epoch;       // single-token decode launch number on this workspace
   unsigned long long theta_word;  // published threshold of token 0 (high word) | flag (low word)
   float theta[8];                 // published thresholds of tokens 1..7

@@ -91,7 +91,7 @@ def source_hash(sources):
     return h.hexdigest()[:16]
 
 
-DECODE_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/ffn_decode.cu",
+DECODE_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/ffn_decode_pg.cu",
                   "activation_sparse_transformer_predictor_b200/csrc/spark_device.cuh"]
 TOPK_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/stat_topk.cu",
                 "activation_sparse_transformer_predictor_b200/csrc/spark_device.cuh"]
@@ -345,10 +345,22 @@ def main():
                 raise _binding.SparkError("spark_ffn_forward", rc)
         return f
 
-    fns = [decode_step(c) for c in copies] * 8  # 128 launches per graph
+    fns = [decode_step(c) for c in copies] * 8  # 128 calls per graph
+    # the score kernel of each call streams its K1 slice while the previous
+    # call's gather kernel runs (programmatic dependent launch)
+    spark.set_weight_overlap(True)
     with ClockSampler(local) as clk:
         ms_step, n_timed = time_graph(fns, args.steps, args.warmup, world)
     ms_step = max_over_ranks(ms_step, world)
+    assert spark.query_status() == 0
+    # the same calls without the overlap, and with the one-launch exchange kernel
+    spark.set_weight_overlap(False)
+    ms_plain, _ = time_graph(fns, min(args.steps, 1280), args.warmup, world)
+    ms_plain = max_over_ranks(ms_plain, world)
+    os.environ["SPARK_DECODE_IMPL"] = "exchange"
+    ms_exch, _ = time_graph(fns, min(args.steps, 1280), args.warmup, world)
+    ms_exch = max_over_ranks(ms_exch, world)
+    del os.environ["SPARK_DECODE_IMPL"]
     assert spark.query_status() == 0
     tok_s = 1e3 / ms_step * world
     achieved_gbs = bytes_per_token / (ms_step * 1e-3) / 1e9
@@ -375,13 +387,22 @@ def main():
     barrier_sync(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
 
-    also = {}
+    also = {
+        "decode_T1_without_weight_overlap": {
+            "tokens_per_s": 1e3 / ms_plain * world, "us_per_call": ms_plain * 1e3,
+            "frac_of_hbm_peak": bytes_per_token / (ms_plain * 1e-3) / 1e9 / hbm_gbs,
+            "note": "score kernel launched after the previous call completes"},
+        "decode_T1_exchange_kernel": {
+            "tokens_per_s": 1e3 / ms_exch * world, "us_per_call": ms_exch * 1e3,
+            "frac_of_hbm_peak": bytes_per_token / (ms_exch * 1e-3) / 1e9 / hbm_gbs,
+            "note": "the alternative one-launch kernel (cooperative, speculative K2 rows, one grid exchange)"},
+    }
     if not args.no_extra:
-        also = extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs)
+        also.update(extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs))
 
     if rank == 0:
         cpu = oracle_baseline(args.cpu_seconds) if world == 1 or rank == 0 else None
-        traffic = profile_traffic("ffn_decode_gemma_T1.txt", DECODE_SOURCES)
+        traffic = profile_traffic("ffn_decode_pg_gemma_T1.txt", DECODE_SOURCES)
         line = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": n_timed,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -392,17 +413,20 @@ def main():
                        "l2": f"inputs larger than L2: steps cycle over {N_COPIES} weight copies "
                              f"({N_COPIES * 2 * D_MODEL * D_FF * 2 / 1e9:.2f} GB)",
                        "timing": "CUDA graph of 128 library calls replayed; CUDA events on the launch stream",
+                       "weight_overlap": "on (spark_set_weight_overlap): each call's score kernel streams K1 "
+                                         "while the previous call's gather kernel runs",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved_gbs / hbm_gbs, "traffic": traffic, "peak_source": peak_src,
-                         "frac_vs_8TBs": achieved_gbs / 8000.0, "kernel": "spark_ffn_decode_kernel",
-                         "duration": "graph replay time per launch (one launch per step, gaps included)",
+                         "frac_vs_8TBs": achieved_gbs / 8000.0,
+                         "kernel": "decode_score_kernel + decode_gather_kernel (one programmatic pair per step)",
+                         "duration": "graph replay time per step (both kernels, gaps included)",
                          "algorithmic_bytes_per_launch": bytes_per_token},
             "cpu_baseline": cpu,
             "e2e": {"value": 1e3 / e2e_ms * world, "unit": "tokens/s", "h2d_bytes_per_step": D_MODEL * 2,
                     "d2h_bytes_per_step": D_MODEL * 2,
                     "path": "public Python API per step: pinned q H2D copy, ffn_forward, out D2H copy"},
-            "gpu_launches": n_timed,
+            "gpu_launches": 2 * n_timed,
             "clocks": clk.summary(),
             "also": also,
         }
@@ -459,8 +483,10 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
                                  "us_per_layer": ms * 1e3 / n_layers,
                                  "achieved_GBs": stack_bytes / (ms * 1e-3) / 1e9,
                                  "frac_of_hbm_peak": stack_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
-                                 "note": "26 distinct layers (2.21 GB of weights > L2), one launch per layer forming "
-                                         "q = RMSNorm(h) in-kernel; bytes counted as K1 + 737 active K2/V rows + q/out per layer"}
+                                 "note": "26 distinct layers (2.21 GB of weights > L2): one score + gather pair per "
+                                         "layer, each layer's K1 streamed under the previous layer's gather; the "
+                                         "gather forms h + out and the next q = RMSNorm(h); bytes counted as K1 + "
+                                         "737 active K2/V rows + q/out per layer"}
     del layers
     # stat top-k on 8 x 4096 x 4096 fp32 rows, k = 256
     rows, d, k = 8 * 4096, 4096, 256

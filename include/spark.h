@@ -155,7 +155,23 @@ SPARK_API double spark_topk_quantile(int k, int d);
  * (grid barriers, copy completions).  Default 1e9 (one second); 0 restores it. */
 SPARK_API int spark_set_wait_limit_ns(unsigned long long ns);
 
-/* Self-test of the bounded waits: launches the decode kernel's grid barrier on
+/*
+ * Single-token decode (spark_ffn_forward, and _tokens / _debug with one token)
+ * runs as two kernels: a score kernel (x, its moments) and a gather kernel
+ * (theta, the active K2 / V rows, out).  With weight overlap enabled (nonzero),
+ * the score kernel is launched as a programmatic dependent of whatever kernel
+ * precedes the call on the stream: it starts streaming K1 into shared memory
+ * while that kernel is still running, and reads q, and writes anything, only
+ * after that kernel has completed.  This hides most of K1's transfer behind the
+ * previous call (or the previous layer) in a decode loop.  The caller promises
+ * that the kernel immediately preceding the call on the stream does not write
+ * K1.  Default 0: the score kernel starts after all earlier work.  Process-wide;
+ * applies to later calls.  spark_ffn_decode_stack always overlaps its own
+ * layers (the kernel ahead of each layer's score kernel is the library's).
+ */
+SPARK_API int spark_set_weight_overlap(int enable);
+
+/* Self-test of the bounded waits: launches the fused kernel's grid barrier on
  * `stream` with an arrival target that can never be met, so that every CTA runs
  * out its time limit and records SPARK_ETIMEOUT.  Call spark_query_status() on
  * the same stream afterwards; it must return SPARK_ETIMEOUT and clears it. */
@@ -171,8 +187,9 @@ SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream);
  * allocate), or a runtime that plans all device memory ahead of time and
  * treats any later allocation as a failure.
  *
- * It computes exactly what spark_ffn_forward computes (one token, same kernel,
- * same arguments, same argument checks) but never calls cudaMalloc,
+ * It computes what spark_ffn_forward computes for one token (same arguments,
+ * same argument checks, same arithmetic up to fp32 summation order; it runs the
+ * single-launch fused kernel that also serves 2-4 tokens) but never calls cudaMalloc,
  * cudaMallocAsync, cudaFree or any allocating library routine.  Its scratch
  * (control block, per-CTA moments, per-CTA partial outputs) lives in one
  * buffer of SPARK_NOALLOC_SCRATCH_BYTES (2 MiB) compiled into the library as a

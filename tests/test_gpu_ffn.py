@@ -170,9 +170,10 @@ def test_bounded_wait_times_out_and_recovers():
 
 @pytest.mark.parametrize("cap", ["0", "3"])
 def test_decode_recompute_path_is_bit_identical(cap, monkeypatch):
-    """The single-token kernel speculates on candidate neurons before theta is known; a CTA
-    whose largest non-candidate score passes theta is recomputed from K1/K2 after the
+    """The one-launch exchange kernel speculates on candidate neurons before theta is known;
+    a CTA whose largest non-candidate score passes theta is recomputed from K1/K2 after the
     exchange.  Forcing few or no speculation slots must give the same bits, and parity."""
+    monkeypatch.setenv("SPARK_DECODE_IMPL", "exchange")
     d_model, r, d_ff, k = GEMMA
     dev, _ = make_layer(d_model, r, d_ff, 1, layer=9)
     q = dev["q"][0].contiguous()
@@ -184,3 +185,64 @@ def test_decode_recompute_path_is_bit_identical(cap, monkeypatch):
     assert torch.equal(forced, ref)
     monkeypatch.setenv("SPARK_DECODE_CAP", cap)
     run_parity(*GEMMA, T=1, layer=9)
+
+
+@pytest.mark.parametrize("cluster", ["4", "2"])
+def test_decode_gather_cluster_sizes(cluster, monkeypatch):
+    """The gather kernel sums its partial outputs through clusters; other cluster sizes
+    change only the fp32 summation order: parity holds for each."""
+    monkeypatch.setenv("SPARK_DECODE_CLUSTER", cluster)
+    run_parity(*GEMMA, T=1, layer=40 + int(cluster))
+    run_parity(*TINY, T=1, layer=41)
+
+
+def test_decode_weight_overlap_in_graph_is_bit_identical():
+    """Score kernels launched behind the previous call (programmatic dependent launch), in a
+    stream and inside a CUDA graph, give the same bits as plain stream order; each call's q
+    is produced by the kernel just before it, so an early read of q would show."""
+    d_model, r, d_ff, k = GEMMA
+    layers = [make_layer(d_model, r, d_ff, 1, layer=60 + i)[0] for i in range(3)]
+    n = 6
+    q0 = layers[0]["q"][0].contiguous()
+
+    def chain(outs):
+        q = q0
+        for i in range(n):
+            L = layers[i % 3]
+            spark.ffn_forward(q, L["K1"], L["K2"], L["V"], k, out=outs[i])
+            q = outs[i]
+
+    ref = [torch.empty(d_model, dtype=torch.bfloat16, device="cuda") for _ in range(n)]
+    spark.set_weight_overlap(False)
+    chain(ref)
+    torch.cuda.synchronize()
+    try:
+        spark.set_weight_overlap(True)
+        got = [torch.empty_like(ref[0]) for _ in range(n)]
+        chain(got)
+        torch.cuda.synchronize()
+        assert all(torch.equal(a, b) for a, b in zip(got, ref))
+        s = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        gout = [torch.empty_like(ref[0]) for _ in range(n)]
+        with torch.cuda.stream(s):
+            chain(gout)  # workspace of this stream exists before capture
+            s.synchronize()
+            with torch.cuda.graph(g, stream=s):
+                chain(gout)
+        for _ in range(3):
+            for t in gout:
+                t.zero_()
+            g.replay()
+            torch.cuda.synchronize()
+            assert all(torch.equal(a, b) for a, b in zip(gout, ref))
+        assert spark.query_status(s) == 0
+    finally:
+        spark.set_weight_overlap(False)
+    assert spark.query_status() == 0
+
+
+def test_decode_exchange_kernel_parity(monkeypatch):
+    """The one-launch exchange kernel (kept as an alternative) stays within parity."""
+    monkeypatch.setenv("SPARK_DECODE_IMPL", "exchange")
+    run_parity(*GEMMA, T=1, layer=50)
