@@ -32,17 +32,13 @@ float g_spec_margin = spec_margin_default();
 // ahead of it on the stream has completed (spark_set_weight_overlap).
 bool g_weight_overlap = false;
 
-// Tuning / test knobs read per call: SPARK_DECODE_IMPL=exchange selects the
-// one-launch exchange kernel instead of the score + gather pair;
-// SPARK_DECODE_CLUSTER forces the gather kernel's cluster size.
+// Tuning / test knob read per call: SPARK_DECODE_IMPL=exchange selects the
+// one-launch exchange kernel instead of the score + gather pair.
 bool decode_use_exchange_kernel() {
   const char* e = std::getenv("SPARK_DECODE_IMPL");
   return e != nullptr && std::strcmp(e, "exchange") == 0;
 }
-int decode_cluster_override() {
-  const char* e = std::getenv("SPARK_DECODE_CLUSTER");
-  return e ? std::atoi(e) : 0;
-}
+
 
 struct DeviceInfo {
   bool probed = false;
@@ -194,7 +190,7 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
   }
 
   if (T == 1 && never_arrive == 0 && !decode_use_exchange_kernel()) {
-    const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin, decode_cluster_override());
+    const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin);
     if (pp.ok) {
       void* ws = nullptr;
       const int wst = get_workspace(dev, stream, pp.ws_bytes, &ws);
@@ -360,17 +356,13 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
   if (dst != SPARK_OK) return dst;
   const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff)));
   if (!decode_use_exchange_kernel()) {
-    const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin, decode_cluster_override());
+    const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin);
     if (!pp.ok) return SPARK_EINVAL;  // shape not supported by the single-token kernels
     void* ws = nullptr;
     const int wst = get_workspace(dev, stream, pp.ws_bytes, &ws);
     if (wst != SPARK_OK) return wst;
-    // q_0 = bf16(RMSNorm(h_0)) into the workspace; every layer's gather kernel
-    // writes h_{l+1} and q_{l+1}
-    if (launch_rmsnorm_q(pp, ws, h_in, d_model, d_ff, eps, stream) != cudaSuccess) {
-      cudaGetLastError();
-      return SPARK_ECUDA;
-    }
+    // every layer's score kernel forms q_l = bf16(RMSNorm(h_l)); its reduce
+    // kernel writes h_{l+1} = h_l + bf16(out_l)
     for (int l = 0; l < n_layers; ++l) {
       DecodePgArgs a;
       a.K1 = K1s[l];
@@ -384,12 +376,12 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
       a.q_dbg = q_dbg ? static_cast<unsigned char*>(q_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
       a.workspace = ws;
       a.wait_limit_ns = g_wait_limit_ns;
-      // the kernel ahead of each score kernel is this library's own (it writes no weights)
-      a.overlap_weights = true;
-      a.q_from_workspace = true;
-      a.h_base = l == 0 ? h_in : h_out;
+      // after the first layer, the kernel ahead of each score kernel is this
+      // library's own reduce kernel, which writes no weights
+      a.overlap_weights = l > 0 || g_weight_overlap;
+      a.h_in = l == 0 ? h_in : h_out;
+      a.h_base = a.h_in;
       a.h_out = h_out;
-      a.write_q_next = l + 1 < n_layers;
       a.eps = eps;
       if (launch_decode_pg(pp, a, stream) != cudaSuccess) {
         cudaGetLastError();

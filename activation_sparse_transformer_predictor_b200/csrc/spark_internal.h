@@ -68,51 +68,42 @@ cudaError_t launch_decode(const DecodePlan& plan, const FusedArgs& args, cudaStr
 
 // ---------------------------------------------------------------- single-token decode: score + gather kernels
 struct DecodePgPlan {
-  int n_slices;           // score-kernel CTAs; slice c = neurons [c*rows_per_cta, ...)
+  int n_slices;           // score- and gather-kernel CTAs; slice c = neurons [c*rows_per_cta, ...)
   int rows_per_cta;       // multiple of 8
-  int slices_per_g;       // score slices handled by one gather CTA
-  int grid_g;             // gather-kernel CTAs (rounded up to the cluster size)
-  int cluster;            // gather-kernel cluster size (8, 4 or 2)
   int chunks_per_thread;  // 16-byte output chunks per gather thread (1, 2 or 4)
   int lane_chunks;        // 16-byte chunks per lane of a K1 / K2 row (5 or 8)
-  int n_clusters;
+  int n_rctas;            // reduce-kernel CTAs (16 output columns each)
   size_t smem_p, smem_g, ws_bytes;
   bool ok;
 };
 
-// cluster_override > 0 forces the gather kernel's cluster size (8, 4, 2).
-DecodePgPlan plan_decode_pg(int d_model, int r, int d_ff, int num_sms, size_t smem_optin, int cluster_override);
+DecodePgPlan plan_decode_pg(int d_model, int r, int d_ff, int num_sms, size_t smem_optin);
 
 struct DecodePgArgs {
-  const void* q = nullptr;  // bf16 [d_model]; ignored when q_from_workspace
+  const void* q = nullptr;      // bf16 [d_model] (ignored when h_in is set)
+  const float* h_in = nullptr;  // stack mode: q = bf16(RMSNorm(h_in)), formed by the score kernel
   const void* K1 = nullptr;
   const void* K2 = nullptr;
   const void* V = nullptr;
-  void* out = nullptr;      // bf16 [d_model]; may be nullptr in stack mode
+  void* out = nullptr;          // bf16 [d_model]; may be nullptr in stack mode
   int d_model = 0, r = 0, d_ff = 0;
   float Q = 0.f;
+  float eps = 0.f;
   float* x_out = nullptr;
   float* theta_out = nullptr;
   unsigned char* active_out = nullptr;
-  void* q_dbg = nullptr;    // bf16 [d_model]: copy of the q used
+  void* q_dbg = nullptr;        // bf16 [d_model]: copy of the q used
   void* workspace = nullptr;
   unsigned long long wait_limit_ns = 0;
   // Launch the score kernel programmatically behind the preceding kernel on the
   // stream: it then reads K1 before that kernel has completed.
   bool overlap_weights = false;
-  // stack mode: q is the workspace q buffer; h_out = h_base + bf16(out) and,
-  // with write_q_next, the q buffer is rewritten with bf16(RMSNorm(h_out))
-  bool q_from_workspace = false;
+  // stack mode, reduce kernel: h_out = h_base + bf16(out) (h_out may equal h_base)
   const float* h_base = nullptr;
   float* h_out = nullptr;
-  bool write_q_next = false;
-  float eps = 0.f;
 };
 
 cudaError_t launch_decode_pg(const DecodePgPlan& plan, const DecodePgArgs& args, cudaStream_t stream);
-// q buffer of the workspace <- bf16(RMSNorm(h)); the stack's first layer reads it.
-cudaError_t launch_rmsnorm_q(const DecodePgPlan& plan, void* workspace, const float* h, int d_model, int d_ff,
-                             float eps, cudaStream_t stream);
 
 // ---------------------------------------------------------------- batched (prefill) FFN on tcgen05
 constexpr int kPrefillMinTokens = kFusedMaxTokens + 1;  // smaller batches take the fused kernel

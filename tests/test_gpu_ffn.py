@@ -187,15 +187,6 @@ def test_decode_recompute_path_is_bit_identical(cap, monkeypatch):
     run_parity(*GEMMA, T=1, layer=9)
 
 
-@pytest.mark.parametrize("cluster", ["4", "2"])
-def test_decode_gather_cluster_sizes(cluster, monkeypatch):
-    """The gather kernel sums its partial outputs through clusters; other cluster sizes
-    change only the fp32 summation order: parity holds for each."""
-    monkeypatch.setenv("SPARK_DECODE_CLUSTER", cluster)
-    run_parity(*GEMMA, T=1, layer=40 + int(cluster))
-    run_parity(*TINY, T=1, layer=41)
-
-
 def test_decode_weight_overlap_in_graph_is_bit_identical():
     """Score kernels launched behind the previous call (programmatic dependent launch), in a
     stream and inside a CUDA graph, give the same bits as plain stream order; each call's q
