@@ -419,8 +419,8 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
                          "frac": achieved_gbs / hbm_gbs, "traffic": traffic, "peak_source": peak_src,
                          "frac_vs_8TBs": achieved_gbs / 8000.0,
-                         "kernel": "decode_score_kernel + decode_gather_kernel (one programmatic pair per step)",
-                         "duration": "graph replay time per step (both kernels, gaps included)",
+                         "kernel": "decode_score_kernel + decode_gather_kernel + decode_reduce_kernel (one programmatic chain per step)",
+                         "duration": "graph replay time per step (three kernels, gaps included)",
                          "algorithmic_bytes_per_launch": bytes_per_token},
             "cpu_baseline": cpu,
             "e2e": {"value": 1e3 / e2e_ms * world, "unit": "tokens/s", "h2d_bytes_per_step": D_MODEL * 2,
