@@ -51,7 +51,8 @@ struct GemmParams {
   int tiles_m, tiles_n, split_k, kb_per_split, nkb, units;
   int nkb0;               // GEMM 2: k-blocks of the first segment (Q1 K1^T); the rest is Q2 K2^T
   float* X;               // optional predictor scores [M][N] written by GEMM 1 (debug)
-  float2* moments;        // [M][tiles_n] (mean, M2) of each 128-neuron tile
+  float2* moments;        // [M][mom_stride] (mean, M2) of each 128-neuron tile
+  int mom_stride;         // 128-neuron tiles per row of moments
   const float* theta;     // [M]
   uint16_t* h_hi;         // [M][N] bf16
   uint16_t* h_lo;         // [M][N] bf16
@@ -148,15 +149,21 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int unit, int& 
   kb1 = min(p.nkb, kb0 + p.kb_per_split);
 }
 
-template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES>
+// WIDE (GEMM 1 only): a unit is 128 rows x 256 columns, two 128-column halves
+// that share the A tile of each stage and own one half of the accumulator each;
+// each k-step issues the same M 128, N 128, K 16 instruction once per half, so
+// every output element sees the instruction sequence of the narrow tile.
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const GemmParams p) {
-  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes;
+  static_assert(!WIDE || (EPI == kEpiPredictor && !B_NMAJOR && !DUAL), "wide units are for GEMM 1");
+  constexpr int kBTiles = WIDE ? 2 : 1;
+  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes * kBTiles;
   // GEMM 2 keeps two accumulators per tile (x and a): two segments of k-blocks
   constexpr bool TWO = EPI == kEpiGate;
-  constexpr int kAccCols = TWO ? 2 * BN : BN;   // TMEM columns of one tile's accumulators
+  constexpr int kAccCols = (TWO || WIDE) ? 2 * BN : BN;   // TMEM columns of one tile's accumulators
   constexpr int kTmemCols = 2 * kAccCols;       // double buffered
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -217,7 +224,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(sb, &tmB, tn * BN, kb * BK, &full[stage]);
             tma_load_2d(sb + kBBytes / 2, &tmB, tn * BN + 64, kb * BK, &full[stage]);
           } else {
-            tma_load_2d(sb, &tmB, kb * BK, tn * BN, &full[stage]);
+#pragma unroll
+            for (int h = 0; h < kBTiles; ++h)
+              tma_load_2d(sb + h * kBBytes, &tmB, kb * BK, (tn * kBTiles + h) * BN, &full[stage]);
           }
         }
         ++issued;
@@ -284,6 +293,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                           : desc_kmajor_sw128(sb + k * 32);
           umma_bf16(d_tmem, desc_kmajor_sw128(sa + k * 32), bdesc, idesc, (!first || k > 0) ? 1u : 0u);
           if (DUAL) umma_bf16(d_tmem, desc_kmajor_sw128(sa + kABytes + k * 32), bdesc, idesc, 1u);
+          if (WIDE)
+            umma_bf16(d_tmem + static_cast<uint32_t>(BN), desc_kmajor_sw128(sa + k * 32),
+                      desc_kmajor_sw128(sb + kBBytes + k * 32), idesc, (!first || k > 0) ? 1u : 0u);
         }
         umma_commit(&empty[stage]);
         if (++stage == STAGES) {
@@ -312,50 +324,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
       const int m = tm * BM + row;
-      const int n_base = tn * BN;
+      const int n_base = tn * BN * kBTiles;
       const bool row_ok = m < p.M;
       float v[16];
       if (EPI == kEpiPredictor) {
         float* xrow = p.X + static_cast<size_t>(m) * p.N;
-        float sum = 0.f;
-        int cnt = 0;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          tmem_ld16(taddr + c, v);
-          const int n = n_base + c;
+        for (int h = 0; h < kBTiles; ++h) {
+          // one 128-column half: moments about its mean (two passes over TMEM)
+          const int nb = n_base + h * BN;
+          const uint32_t ta = taddr + static_cast<uint32_t>(h * BN);
+          float sum = 0.f;
+          int cnt = 0;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 16) {
+            tmem_ld16(ta + c, v);
+            const int n = nb + c;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (n + j < p.N) {
-              sum += v[j];
-              ++cnt;
-            }
-          if (row_ok && p.X != nullptr) {
-            if (n + 16 <= p.N) {
-              float4* d = reinterpret_cast<float4*>(xrow + n);
-              d[0] = make_float4(v[0], v[1], v[2], v[3]);
-              d[1] = make_float4(v[4], v[5], v[6], v[7]);
-              d[2] = make_float4(v[8], v[9], v[10], v[11]);
-              d[3] = make_float4(v[12], v[13], v[14], v[15]);
-            } else {
-              for (int j = 0; j < 16; ++j)
-                if (n + j < p.N) xrow[n + j] = v[j];
+            for (int j = 0; j < 16; ++j)
+              if (n + j < p.N) {
+                sum += v[j];
+                ++cnt;
+              }
+            if (row_ok && p.X != nullptr) {
+              if (n + 16 <= p.N) {
+                float4* d = reinterpret_cast<float4*>(xrow + n);
+                d[0] = make_float4(v[0], v[1], v[2], v[3]);
+                d[1] = make_float4(v[4], v[5], v[6], v[7]);
+                d[2] = make_float4(v[8], v[9], v[10], v[11]);
+                d[3] = make_float4(v[12], v[13], v[14], v[15]);
+              } else {
+                for (int j = 0; j < 16; ++j)
+                  if (n + j < p.N) xrow[n + j] = v[j];
+              }
             }
           }
-        }
-        const float mean = cnt > 0 ? sum / static_cast<float>(cnt) : 0.f;
-        float m2 = 0.f;
+          const float mean = cnt > 0 ? sum / static_cast<float>(cnt) : 0.f;
+          float m2 = 0.f;
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          tmem_ld16(taddr + c, v);
-          const int n = n_base + c;
+          for (int c = 0; c < BN; c += 16) {
+            tmem_ld16(ta + c, v);
+            const int n = nb + c;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (n + j < p.N) {
-              const float d = v[j] - mean;
-              m2 += d * d;
-            }
+            for (int j = 0; j < 16; ++j)
+              if (n + j < p.N) {
+                const float d = v[j] - mean;
+                m2 += d * d;
+              }
+          }
+          if (row_ok && nb < p.N) p.moments[static_cast<size_t>(m) * p.mom_stride + nb / BN] = make_float2(mean, m2);
         }
-        if (row_ok) p.moments[static_cast<size_t>(m) * p.tiles_n + tn] = make_float2(mean, m2);
       } else if (EPI == kEpiGate) {
         const float th = row_ok ? p.theta[m] : 0.f;
 #pragma unroll 1
@@ -540,12 +558,12 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES>
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const CUtensorMap& b2,
                         const GemmParams& p, int num_sms, cudaStream_t stream) {
-  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes;
+  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes * (WIDE ? 2 : 1);
   constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256;
-  auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES>;
+  auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE>;
   static int set_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -614,6 +632,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   g.wait_limit_ns = a.wait_limit_ns;
   g.X = a.x_out;  // scores leave the chip only for the debug entry point
   g.moments = moments;
+  g.mom_stride = tiles_n;
   g.theta = theta;
   g.h_hi = h_hi;
   g.h_lo = h_lo;
@@ -631,11 +650,23 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   g.split_k = 1;
   g.kb_per_split = g.nkb;
   g.units = g.tiles_m * g.tiles_n;
-  cudaError_t e = launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  // Wide units (128 tokens x 256 neurons, 4 stages of 48 KB) carry twice the MMA
+  // work per token tile loaded; they pay off once they still fill every SM.
+  const int wide_units = g.tiles_m * ((d_ff + 2 * BN - 1) / (2 * BN));
+  cudaError_t e;
+  if (wide_units >= num_sms) {
+    g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
+    g.units = wide_units;
+    e = launch_gemm<kEpiPredictor, false, false, 4, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  } else {
+    e = launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  }
   if (e != cudaSuccess) return e;
   theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, tiles_n, a.Q, theta, a.theta_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // GEMM 2: X = Q1 K1^T again and A = Q2 K2^T, gate and split
+  // GEMM 2: X = Q1 K1^T again and A = Q2 K2^T, gate and split (narrow units)
+  g.tiles_n = tiles_n;
+  g.units = g.tiles_m * g.tiles_n;
   g.K = d_model;
   g.nkb0 = (r + BK - 1) / BK;
   g.nkb = g.nkb0 + (d2 + BK - 1) / BK;

@@ -83,6 +83,16 @@ def test_gemma_prefill_large_sampled(T):
     run_parity(*GEMMA, T=T, layer=30 + T, sample_tokens=sample)
 
 
+def test_prefill_wide_predictor_ragged_last_unit():
+    """Enough tokens for the predictor GEMM's 128 x 256 units, with d_ff = 2496 so that the last
+    unit's second 128-column half is only half inside the layer."""
+    T = 1920
+    rng = np.random.default_rng(7)
+    sample = np.sort(rng.choice(T, size=16, replace=False))
+    sample[0], sample[-1] = 0, T - 1
+    run_parity(512, 256, 2496, 200, T=T, layer=77, sample_tokens=sample)
+
+
 @pytest.mark.parametrize("shape", [
     (264, 136, 1001, 80, 3),    # ragged d_ff: last CTA owns one neuron
     (64, 32, 200, 17, 2),       # tiny, few CTAs
