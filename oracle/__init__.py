@@ -72,6 +72,12 @@ def _load():
         lib.oracle_spark_ffn.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_long] * 5 + [
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_softplus.restype = ctypes.c_double
+        lib.oracle_softplus.argtypes = [ctypes.c_double]
+        lib.oracle_spark_attention.restype = ctypes.c_int
+        lib.oracle_spark_attention.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_long] * 6 + [
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int]
         lib.oracle_rmsnorm.restype = None
         lib.oracle_rmsnorm.argtypes = [dp, ctypes.c_long, ctypes.c_double, dp]
         lib.oracle_num_threads_available.restype = ctypes.c_int
@@ -187,3 +193,37 @@ def rmsnorm(h: np.ndarray, eps: float = 1e-6) -> np.ndarray:
     y = np.empty_like(h)
     _load().oracle_rmsnorm(_dptr(h), h.size, float(eps), _dptr(y))
     return y
+
+
+def softplus(a: float) -> float:
+    return float(_load().oracle_softplus(float(a)))
+
+
+def spark_attention(q_bits, K_bits, V_bits, r: int, k_attn: int, scale: float, override_active=None,
+                    n_threads: int = 1):
+    """Spark Attention for one decoding position on bf16 bit patterns (uint16 arrays).
+
+    q_bits [n_heads, d_head]; K_bits and V_bits [n_kv_heads, n_ctx, d_head].  Returns a dict with
+    out [n_heads, d_head] (fp64), s [n_heads, n_ctx] (scaled predictor scores), theta [n_heads]
+    (-inf when every key is selected) and active [n_heads, n_ctx] (bool, s > theta).
+    """
+    q = np.ascontiguousarray(q_bits, dtype=np.uint16)
+    K = np.ascontiguousarray(K_bits, dtype=np.uint16)
+    V = np.ascontiguousarray(V_bits, dtype=np.uint16)
+    n_heads, d_head = q.shape
+    n_kv, n_ctx, dk = K.shape
+    if dk != d_head or V.shape != K.shape or n_heads % n_kv != 0:
+        raise ValueError("oracle.spark_attention: inconsistent shapes")
+    ov = None
+    if override_active is not None:
+        ov = np.ascontiguousarray(override_active, dtype=np.uint8).reshape(n_heads, n_ctx)
+    out = np.empty((n_heads, d_head), dtype=np.float64)
+    sc = np.empty((n_heads, n_ctx), dtype=np.float64)
+    th = np.empty(n_heads, dtype=np.float64)
+    act = np.empty((n_heads, n_ctx), dtype=np.uint8)
+    rc = _load().oracle_spark_attention(_ptr(q), _ptr(K), _ptr(V), n_heads, n_kv, n_ctx, d_head, int(r),
+                                        int(k_attn), float(scale), _ptr(ov), _ptr(out), _ptr(sc), _ptr(th),
+                                        _ptr(act), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_spark_attention: invalid arguments")
+    return {"out": out, "s": sc, "theta": th, "active": act.astype(bool)}

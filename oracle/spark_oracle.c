@@ -28,7 +28,11 @@
  * exactly); sums run in plain index order; no blocking, fusion or reordering.
  * Build with -ffp-contract=off so that a*b+c is never fused.
  *
- * parity pins: see tests/test_oracle_pins.py (sorted top-m, closed-form theta,
+ * Spark Attention (one decoding position) follows the same page, item "Spark
+ * Attention"; its readings are at oracle_spark_attention.
+ *
+ * parity pins: see tests/test_oracle_pins.py and tests/test_oracle_attention_pins.py
+ * (sorted top-m, closed-form theta,
  * textbook quantiles, GELU vs x*Phi(x), invariants, degenerate rows, reduction
  * of the FFN to GELU(SoftThreshold) for identity-like K2/V).
  */
@@ -210,6 +214,92 @@ int oracle_spark_ffn(const uint16_t *q, const uint16_t *K1, const uint16_t *K2,
         if (mean_out) mean_out[t] = mean;
         if (std_out) std_out[t] = sd;
         free(x);
+    }
+    return 0;
+}
+
+/* softplus(a) = log(1 + e^a), evaluated without overflow. */
+double oracle_softplus(double a)
+{
+    return a > 0.0 ? a + log1p(exp(-a)) : log1p(exp(a));
+}
+
+/*
+ * Spark Attention for one decoding position ("Spark Attention" in 关键设计): the
+ * key vectors are split like the FFN's K into K1 (the first r dimensions, used
+ * to predict) and K2 (the rest); each query attends to at most k_attn keys
+ * chosen by statistical top-k on the predictor scores; sigma_1 = softmax and
+ * sigma_2 = softplus.  For query head h (key/value head g = h / (n_heads /
+ * n_kv_heads)):
+ *   s_j   = scale * sum_{i<r} K[g][j][i] q[h][i]                (j < n_ctx)
+ *   theta = mean(s) + std(s) Q(1 - k_attn/n_ctx); A = { j : s_j > theta }
+ *           (k_attn >= n_ctx: every key, the min{k_attn, n_ctx} of the FLOP count)
+ *   p_j   = exp(s_j) / sum_{l in A} exp(s_l)                       (j in A)
+ *   a_j   = sum_{i<d_head-r} K[g][j][r+i] q[h][r+i]
+ *   out[h] = sum_{j in A} p_j softplus(a_j) V[g][j][:]
+ * Readings: the softmax runs over the selected keys only (a softmax over all
+ * n_ctx soft-thresholded scores would give every unselected key the weight
+ * e^0 and attend densely); softmax is shift-invariant, so it is the same on s_j
+ * and on the soft-thresholded s_j - theta; `scale` is the attention temperature,
+ * which the page leaves open (callers pass 1/sqrt(d_head) by default); an
+ * empty A (zero spread) gives out = 0.
+ * Layouts: q [n_heads][d_head], K and V [n_kv_heads][n_ctx][d_head] bf16 bits;
+ * out fp64 [n_heads][d_head].  s_out [n_heads][n_ctx], theta_out [n_heads],
+ * active_out [n_heads][n_ctx] are optional; override_active ([n_heads][n_ctx])
+ * replaces A (the weights are then renormalised over the given set).
+ * Returns 0, or -1 on invalid sizes.
+ */
+int oracle_spark_attention(const uint16_t *q, const uint16_t *K, const uint16_t *V, long n_heads,
+                           long n_kv_heads, long n_ctx, long d_head, long r, long k_attn, double scale,
+                           const uint8_t *override_active, double *out, double *s_out, double *theta_out,
+                           uint8_t *active_out, int n_threads)
+{
+    if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0 || n_ctx < 1 || !(r > 0 && r < d_head) ||
+        k_attn < 1)
+        return -1;
+    if (n_threads < 1) n_threads = 1;
+    const long group = n_heads / n_kv_heads;
+#pragma omp parallel for schedule(static) num_threads(n_threads)
+    for (long h = 0; h < n_heads; ++h) {
+        const long g = h / group;
+        const uint16_t *qh = q + h * d_head;
+        const uint16_t *Kg = K + g * n_ctx * d_head;
+        const uint16_t *Vg = V + g * n_ctx * d_head;
+        double *s = (double *)malloc(sizeof(double) * (size_t)n_ctx);
+        for (long j = 0; j < n_ctx; ++j) {
+            double acc = 0.0;
+            for (long i = 0; i < r; ++i)
+                acc += oracle_bf16_to_f64(Kg[j * d_head + i]) * oracle_bf16_to_f64(qh[i]);
+            s[j] = scale * acc;
+        }
+        double theta = -INFINITY;
+        if (k_attn < n_ctx) theta = oracle_theta(s, n_ctx, k_attn, NULL, NULL);
+        double smax = -INFINITY;
+        for (long j = 0; j < n_ctx; ++j) {
+            int act = override_active ? (override_active[h * n_ctx + j] != 0) : (s[j] > theta);
+            if (active_out) active_out[h * n_ctx + j] = (uint8_t)(s[j] > theta);
+            if (act && s[j] > smax) smax = s[j];
+        }
+        double *o = out + h * d_head;
+        for (long c = 0; c < d_head; ++c) o[c] = 0.0;
+        double z = 0.0;
+        for (long j = 0; j < n_ctx; ++j) {
+            int act = override_active ? (override_active[h * n_ctx + j] != 0) : (s[j] > theta);
+            if (!act) continue;
+            double w = exp(s[j] - smax);
+            double a = 0.0;
+            for (long i = 0; i < d_head - r; ++i)
+                a += oracle_bf16_to_f64(Kg[j * d_head + r + i]) * oracle_bf16_to_f64(qh[r + i]);
+            double f = w * oracle_softplus(a);
+            for (long c = 0; c < d_head; ++c) o[c] += f * oracle_bf16_to_f64(Vg[j * d_head + c]);
+            z += w;
+        }
+        if (z > 0.0)
+            for (long c = 0; c < d_head; ++c) o[c] /= z;
+        if (s_out)
+            for (long j = 0; j < n_ctx; ++j) s_out[h * n_ctx + j] = s[j];
+        if (theta_out) theta_out[h] = theta;
+        free(s);
     }
     return 0;
 }

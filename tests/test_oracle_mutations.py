@@ -30,6 +30,44 @@ MUTATIONS = {
 }
 
 
+# Mistakes planted in the Spark Attention oracle; the attention pins must catch each.
+ATTN_MUTATIONS = {
+    "attn_scale_dropped": ("s[j] = scale * acc;", "s[j] = acc;"),
+    "attn_softplus_sign": ("return a > 0.0 ? a + log1p(exp(-a)) : log1p(exp(a));",
+                           "return a > 0.0 ? a - log1p(exp(-a)) : log1p(exp(a));"),
+    "attn_a_uses_predictor_dims": ("a += oracle_bf16_to_f64(Kg[j * d_head + r + i]) * oracle_bf16_to_f64(qh[r + i]);",
+                                   "a += oracle_bf16_to_f64(Kg[j * d_head + i]) * oracle_bf16_to_f64(qh[i]);"),
+    "attn_no_normalisation": ("for (long c = 0; c < d_head; ++c) o[c] /= z;",
+                              "for (long c = 0; c < d_head; ++c) o[c] /= 1.0;"),
+    "attn_wrong_kv_head": ("const long g = h / group;", "const long g = h % n_kv_heads;"),
+    "attn_theta_ignored": ("if (k_attn < n_ctx) theta = oracle_theta(s, n_ctx, k_attn, NULL, NULL);", ""),
+    "attn_value_from_key": ("o[c] += f * oracle_bf16_to_f64(Vg[j * d_head + c]);",
+                            "o[c] += f * oracle_bf16_to_f64(Kg[j * d_head + c]);"),
+}
+
+
+def _pins_fail_on(old, new, pin_file, tmp_path):
+    src = open(SRC).read()
+    assert src.count(old) == 1, "mutation anchor not found exactly once"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-D_GNU_SOURCE", "-ffp-contract=off", "-fopenmp",
+                           "-fPIC", "-shared", str(mutated), "-o", str(lib), "-lm"])
+    env = dict(os.environ, SPARK_ORACLE_LIB=str(lib))
+    proc = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                           os.path.join(ROOT, "tests", pin_file)],
+                          env=env, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    return proc.returncode != 0, proc.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name", sorted(ATTN_MUTATIONS))
+def test_attention_pins_catch_planted_mistake(name, tmp_path):
+    old, new = ATTN_MUTATIONS[name]
+    caught, log = _pins_fail_on(old, new, "test_oracle_attention_pins.py", tmp_path)
+    assert caught, f"attention pins did not catch mutation {name}:\n{log}"
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_pins_catch_planted_mistake(name, tmp_path):
     old, new = MUTATIONS[name]
