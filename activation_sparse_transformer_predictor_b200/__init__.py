@@ -146,6 +146,47 @@ def set_wait_limit_ns(ns: int) -> None:
     _binding.check("spark_set_wait_limit_ns", _binding.lib().spark_set_wait_limit_ns(int(ns)))
 
 
+def attention_decode(q, K, V, r: int, k_attn: int, scale: float | None = None, out=None, debug: bool = False,
+                     stream=None):
+    """Spark Attention for one decoding position (spark_attention_decode).
+
+    q: bf16 [n_heads, d_head]; K, V: bf16 [n_kv_heads, n_ctx, d_head].  scale defaults to
+    1/sqrt(d_head).  Returns out (bf16 [n_heads, d_head]), or with debug=True a dict with out,
+    s (fp32 [n_heads, n_ctx]), theta (fp32 [n_heads]) and active (uint8 [n_heads, n_ctx]).
+    """
+    import math
+
+    import torch
+    _require(q, "q", torch.bfloat16, (2,))
+    _require(K, "K", torch.bfloat16, (3,))
+    _require(V, "V", torch.bfloat16, (3,))
+    n_heads, d_head = q.shape
+    n_kv, n_ctx, dk = K.shape
+    if dk != d_head or tuple(V.shape) != tuple(K.shape):
+        raise ValueError("attention_decode: q [H, d], K and V [H_kv, n_ctx, d]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d_head)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _require(out, "out", torch.bfloat16, (2,))
+    st = _binding.stream_handle(stream)
+    L = _binding.lib()
+    if not debug:
+        rc = L.spark_attention_decode(q.data_ptr(), K.data_ptr(), V.data_ptr(), n_heads, n_kv, n_ctx, d_head,
+                                      int(r), int(k_attn), float(scale), out.data_ptr(), st)
+        _binding.check("spark_attention_decode", rc)
+        return out
+    s = torch.empty((n_heads, n_ctx), dtype=torch.float32, device=q.device)
+    th = torch.empty(n_heads, dtype=torch.float32, device=q.device)
+    act = torch.empty((n_heads, n_ctx), dtype=torch.uint8, device=q.device)
+    rc = L.spark_attention_decode_debug(q.data_ptr(), K.data_ptr(), V.data_ptr(), n_heads, n_kv, n_ctx, d_head,
+                                        int(r), int(k_attn), float(scale), out.data_ptr(), s.data_ptr(),
+                                        th.data_ptr(), act.data_ptr(), st)
+    _binding.check("spark_attention_decode_debug", rc)
+    return {"out": out, "s": s, "theta": th, "active": act}
+
+
 def set_weight_overlap(enable: bool) -> None:
     """Let the single-token score kernel stream K1 behind the preceding kernel (spark_set_weight_overlap)."""
     _binding.check("spark_set_weight_overlap", _binding.lib().spark_set_weight_overlap(1 if enable else 0))

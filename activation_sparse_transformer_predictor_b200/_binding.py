@@ -23,7 +23,8 @@ STATUS_NAMES = {0: "SPARK_OK", -1: "SPARK_EINVAL", -2: "SPARK_EALIGN", -3: "SPAR
 EXPORTS = ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug", "stat_topk_soft_threshold",
            "spark_query_status", "spark_release_workspace", "spark_status_string", "spark_topk_quantile",
            "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc",
-           "spark_ffn_decode_stack", "spark_set_weight_overlap")
+           "spark_ffn_decode_stack", "spark_set_weight_overlap", "spark_attention_decode",
+           "spark_attention_decode_debug")
 
 _lock = threading.Lock()
 _lib = None
@@ -58,6 +59,9 @@ def lib() -> ctypes.CDLL:
         L.spark_topk_quantile.restype = ctypes.c_double
         L.spark_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
         L.spark_set_weight_overlap.argtypes = [ci]
+        L.spark_attention_decode.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, ctypes.c_float, vp, vp]
+        L.spark_attention_decode_debug.argtypes = [vp, vp, vp, ci, ci, ci, ci, ci, ci, ctypes.c_float, vp, vp, vp,
+                                                   vp, vp]
         L.spark_selftest_wait_timeout.argtypes = [vp]
         L.spark_version.argtypes = []
         L.spark_ffn_forward_noalloc.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
@@ -65,7 +69,8 @@ def lib() -> ctypes.CDLL:
         for name in ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug",
                      "stat_topk_soft_threshold", "spark_query_status", "spark_release_workspace",
                      "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc",
-                     "spark_ffn_decode_stack", "spark_set_weight_overlap"):
+                     "spark_ffn_decode_stack", "spark_set_weight_overlap", "spark_attention_decode",
+                     "spark_attention_decode_debug"):
             getattr(L, name).restype = ci
         _lib = L
         return L

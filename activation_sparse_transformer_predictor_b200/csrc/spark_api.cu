@@ -429,6 +429,56 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
   return SPARK_OK;
 }
 
+SPARK_API int spark_attention_decode_debug(const void* q, const void* K, const void* V, int n_heads, int n_kv_heads,
+                                          int n_ctx, int d_head, int r, int k_attn, float scale, void* out,
+                                          float* s_out, float* theta_out, unsigned char* active_out,
+                                          spark_stream_t stream) {
+  if (!q || !K || !V || !out) return SPARK_EINVAL;
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads != 0 || n_ctx < 1 || n_ctx > 65536 || k_attn < 1)
+    return SPARK_EINVAL;
+  if (!(r > 0 && r < d_head) || d_head > kAttnMaxDHead) return SPARK_EINVAL;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return SPARK_EINVAL;
+  if (r % 8 != 0 || d_head % 8 != 0) return SPARK_EALIGN;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(out)) return SPARK_EALIGN;
+  const size_t ob = static_cast<size_t>(n_heads) * d_head * 2;
+  const size_t kvb = static_cast<size_t>(n_kv_heads) * n_ctx * d_head * 2;
+  if (overlaps(out, ob, q, ob) || overlaps(out, ob, K, kvb) || overlaps(out, ob, V, kvb)) return SPARK_EINVAL;
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  AttnArgs a;
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.out = out;
+  a.n_heads = n_heads;
+  a.n_kv_heads = n_kv_heads;
+  a.n_ctx = n_ctx;
+  a.d_head = d_head;
+  a.r = r;
+  a.scale = scale;
+  a.select_all = k_attn >= n_ctx;
+  a.Q = a.select_all ? 0.f
+                     : static_cast<float>(upper_tail_quantile(static_cast<double>(k_attn) / static_cast<double>(n_ctx)));
+  a.s_out = s_out;
+  a.theta_out = theta_out;
+  a.active_out = active_out;
+  if (launch_attn_decode(a, di.num_sms, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return SPARK_OK;
+}
+
+SPARK_API int spark_attention_decode(const void* q, const void* K, const void* V, int n_heads, int n_kv_heads,
+                                    int n_ctx, int d_head, int r, int k_attn, float scale, void* out,
+                                    spark_stream_t stream) {
+  return spark_attention_decode_debug(q, K, V, n_heads, n_kv_heads, n_ctx, d_head, r, k_attn, scale, out, nullptr,
+                                      nullptr, nullptr, stream);
+}
+
 SPARK_API int stat_topk_soft_threshold(const float* x, int rows, int d, int k, float* out, spark_stream_t stream) {
   if (rows == 0) return SPARK_OK;
   if (!x || !out || rows < 0 || d < 2 || !(k > 0 && k < d)) return SPARK_EINVAL;

@@ -105,6 +105,25 @@ struct DecodePgArgs {
 
 cudaError_t launch_decode_pg(const DecodePgPlan& plan, const DecodePgArgs& args, cudaStream_t stream);
 
+// ---------------------------------------------------------------- Spark Attention, one decoding position
+constexpr int kAttnMaxDHead = 256;
+constexpr int kAttnMaxKeysPerCta = 2048;
+
+struct AttnArgs {
+  const void* q = nullptr;  // bf16 [n_heads][d_head]
+  const void* K = nullptr;  // bf16 [n_kv_heads][n_ctx][d_head]
+  const void* V = nullptr;  // bf16 [n_kv_heads][n_ctx][d_head]
+  void* out = nullptr;      // bf16 [n_heads][d_head]
+  int n_heads = 0, n_kv_heads = 0, n_ctx = 0, d_head = 0, r = 0;
+  float scale = 1.f, Q = 0.f;
+  bool select_all = false;  // k_attn >= n_ctx
+  float* s_out = nullptr;
+  float* theta_out = nullptr;
+  unsigned char* active_out = nullptr;
+};
+
+cudaError_t launch_attn_decode(const AttnArgs& args, int num_sms, cudaStream_t stream);
+
 // ---------------------------------------------------------------- batched (prefill) FFN on tcgen05
 constexpr int kPrefillMinTokens = kFusedMaxTokens + 1;  // smaller batches take the fused kernel
 

@@ -12,8 +12,11 @@ are not available):
 * tokens q: ``randn`` fp32 -> bf16, i.e. ~N(0, 1).
 * score rows: fp32 ~N(0, 1), or Student-t with 4 degrees of freedom drawn as
   Z / sqrt(W / 4) with W = -2 ln(U1 U2) ~ chi-square(4).
+* attention (one decoding position): query heads, cached keys and values
+  ``randn`` fp32 -> bf16, i.e. ~N(0, 1) (a random model's KV cache).
 * seeds: every tensor has its own ``torch.Generator`` seeded with
-  ``(base + layer) * 8 + slot`` (slot 0 = K1, 1 = K2, 2 = V, 3 = q, 4 = scores).
+  ``(base + layer) * 8 + slot`` (slot 0 = K1, 1 = K2, 2 = V, 3 = q, 4 = scores,
+  5 = residual, 6 = attention keys, 7 = attention values; attention queries use slot 3).
 """
 from __future__ import annotations
 
@@ -22,7 +25,7 @@ import math
 import torch
 
 BASE_SEED = 1234
-_SLOT = {"K1": 0, "K2": 1, "V": 2, "q": 3, "scores": 4, "h": 5}
+_SLOT = {"K1": 0, "K2": 1, "V": 2, "q": 3, "scores": 4, "h": 5, "keys": 6, "values": 7}
 
 
 def _gen(slot: str, layer: int = 0, base: int = BASE_SEED) -> torch.Generator:
@@ -66,6 +69,15 @@ def score_rows(rows: int, d: int, dist: str = "normal", base: int = BASE_SEED) -
         w = -2.0 * torch.log(u1 * u2)
         return (z.double() / torch.sqrt(w / 4.0)).float().contiguous()
     raise ValueError(f"unknown distribution {dist!r}")
+
+
+def attention_inputs(n_heads: int, n_kv_heads: int, n_ctx: int, d_head: int, layer: int = 0,
+                     base: int = BASE_SEED) -> dict:
+    """q [n_heads, d_head], K and V [n_kv_heads, n_ctx, d_head], all bf16 ~N(0, 1)."""
+    q = _randn((n_heads, d_head), _gen("q", layer, base)).to(torch.bfloat16)
+    K = _randn((n_kv_heads, n_ctx, d_head), _gen("keys", layer, base)).to(torch.bfloat16)
+    V = _randn((n_kv_heads, n_ctx, d_head), _gen("values", layer, base)).to(torch.bfloat16)
+    return {"q": q, "K": K, "V": V}
 
 
 def bf16_bits(t: torch.Tensor):

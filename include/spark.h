@@ -122,6 +122,40 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
                                      void* out_dbg, spark_stream_t stream);
 
 /*
+ * Spark Attention for one decoding position (the page's "Spark Attention": the
+ * key vectors split into a predictor part K1 = K[:, :r] and K2 = K[:, r:];
+ * statistical top-k over the predictor scores with k_attn keys per query;
+ * sigma_1 = softmax, sigma_2 = softplus).  For query head h and its key/value
+ * head g = h / (n_heads / n_kv_heads):
+ *   s_j    = scale * <K[g][j][:r], q[h][:r]>                      (j < n_ctx)
+ *   theta  = mean(s) + std(s) * Q(1 - k_attn/n_ctx)   (population std; when
+ *            k_attn >= n_ctx every key is selected)
+ *   out[h] = sum_{s_j > theta} softmax_j(s) * softplus(<K[g][j][r:], q[h][r:]>) * V[g][j][:]
+ * with the softmax over the selected keys only (readings: the page names the
+ * two functions but not where the softmax runs; over all keys it would attend
+ * densely).  An empty selection (zero spread) gives out[h] = 0.
+ *   q    : bf16 [n_heads][d_head]
+ *   K, V : bf16 [n_kv_heads][n_ctx][d_head] (row-major, one row per cached position)
+ *   out  : bf16 [n_heads][d_head]; must not overlap q, K or V
+ *   scale: the attention temperature (> 0, finite), e.g. 1/sqrt(d_head)
+ * Requires n_heads % n_kv_heads == 0, 1 <= n_ctx <= 65536, k_attn >= 1,
+ * 0 < r < d_head <= 256 with r and d_head multiples of 8 (else SPARK_EINVAL /
+ * SPARK_EALIGN), and 16-byte aligned pointers.  One launch; needs no workspace.
+ */
+SPARK_API int spark_attention_decode(const void* q, const void* K, const void* V, int n_heads, int n_kv_heads,
+                                    int n_ctx, int d_head, int r, int k_attn, float scale, void* out,
+                                    spark_stream_t stream);
+
+/* spark_attention_decode, also returning (any may be NULL): s_out fp32
+ * [n_heads][n_ctx] (scaled predictor scores), theta_out fp32 [n_heads]
+ * (-inf when every key is selected), active_out bytes [n_heads][n_ctx]
+ * (1 where s > theta). */
+SPARK_API int spark_attention_decode_debug(const void* q, const void* K, const void* V, int n_heads, int n_kv_heads,
+                                          int n_ctx, int d_head, int r, int k_attn, float scale, void* out,
+                                          float* s_out, float* theta_out, unsigned char* active_out,
+                                          spark_stream_t stream);
+
+/*
  * Standalone statistical top-k with soft threshold ("Statistical Top-k"):
  * for every row of x (fp32 [rows][d]), theta = mean + std * Q(1 - k/d) and
  * out = max(x - theta, 0) (fp32 [rows][d]).  out may equal x (in place); any
