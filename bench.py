@@ -487,11 +487,39 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
                                  "us_per_layer": ms * 1e3 / n_layers,
                                  "achieved_GBs": stack_bytes / (ms * 1e-3) / 1e9,
                                  "frac_of_hbm_peak": stack_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
-                                 "note": "26 distinct layers (2.21 GB of weights > L2): one score + gather pair per "
-                                         "layer, each layer's K1 streamed under the previous layer's gather; the "
-                                         "gather forms h + out and the next q = RMSNorm(h); bytes counted as K1 + "
-                                         "737 active K2/V rows + q/out per layer"}
+                                 "note": "26 distinct layers (2.21 GB of weights > L2): one score, gather and reduce "
+                                         "kernel per layer, each layer's K1 streamed under the previous layer's "
+                                         "gather and reduce; the reduce kernel writes h + out and the next score "
+                                         "kernel forms q = RMSNorm(h); bytes counted as K1 + 737 active K2/V rows + "
+                                         "q/out per layer"}
     del layers
+    # Spark Attention, one decoding position: 8 query heads over 4 key/value heads, d_head 256 split
+    # r = 128, 4096 cached positions, k_attn = 256 (Gemma-2-2B-like heads), 16 distinct caches cycled
+    import math as _m
+    H, KV, NC, DH, RA, KA = 8, 4, 4096, 256, 128, 256
+    caches = []
+    for c in range(16):
+        host = synthetic.attention_inputs(H, KV, NC, DH, layer=c)
+        caches.append({n: t.to(dev) for n, t in host.items()})
+    aout = torch.empty_like(caches[0]["q"])
+
+    def attn(c):
+        def f():
+            rc = L.spark_attention_decode(c["q"].data_ptr(), c["K"].data_ptr(), c["V"].data_ptr(), H, KV, NC, DH, RA,
+                                          KA, 1.0 / _m.sqrt(DH), aout.data_ptr(), _binding.stream_handle())
+            if rc != 0:
+                raise _binding.SparkError("spark_attention_decode", rc)
+        return f
+
+    ms, n = time_graph([attn(c) for c in caches] * 4, 640, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    abytes = KV * NC * RA * 2 + H * KA * ((DH - RA) + DH) * 2 + 2 * H * DH * 2
+    res["spark_attention_decode_8x4096"] = {
+        "calls_per_s": 1e3 / ms * world, "us_per_call": ms * 1e3, "achieved_GBs": abytes / (ms * 1e-3) / 1e9,
+        "frac_of_hbm_peak": abytes / (ms * 1e-3) / 1e9 / hbm_gbs, "algorithmic_bytes_per_call": abytes,
+        "note": "one launch, one 16-CTA cluster per query head; bytes = predictor parts of all cached keys + "
+                "K2 parts and value rows of ~256 selected keys per head + q/out; 16 caches (75 MB) cycled"}
+    del caches
     # stat top-k on 8 x 4096 x 4096 fp32 rows, k = 256
     rows, d, k = 8 * 4096, 4096, 256
     xs = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))

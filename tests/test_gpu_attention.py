@@ -122,3 +122,10 @@ def test_repeatable_and_errors_refused():
                                     out.data_ptr(), st) == -1
     assert L.spark_attention_decode(q.data_ptr(), K.data_ptr(), V.data_ptr(), 8, 4, 2048, 256, 12, 128, 0.0625,
                                     out.data_ptr(), st) == -2
+
+
+def test_portable_cluster_size(monkeypatch):
+    """The 8-CTA cluster path (used where 16-CTA clusters are unavailable) keeps parity."""
+    monkeypatch.setenv("SPARK_ATTN_CLUSTER", "8")
+    run_attention(8, 4, 4096, 256, 128, 256, layer=8)
+    run_attention(2, 1, 1000, 128, 64, 100, layer=9)
