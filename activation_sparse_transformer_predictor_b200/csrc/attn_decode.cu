@@ -13,18 +13,24 @@
 // One thread-block cluster per query head (CS CTAs, distributed shared memory),
 // one launch, no global exchange: every dependency stays inside the cluster.
 //  scores   CTA q of the cluster scores keys [q*KPC, (q+1)*KPC): per key, a group
-//           of lanes reads the K1 part in 16-byte chunks (eight keys in flight
-//           per lane) and reduces with shuffles.
-//  stats    the CTA's (count, mean, M2, max), two passes over shared memory;
-//           cluster barrier; every CTA merges the CS records in rank order, so
-//           all derive the same bits of theta and of the score maximum M.
-//  gather   the selected keys of the CTA: a = <K2[j], q[r:]> (one warp per key),
-//           w = exp(s_j - M), f = w softplus(a); the CTA's partial numerator
-//           sum f_j V[j] (thread groups over keys, fixed-order reduction) and
-//           partial normaliser sum w_j.
-//  reduce   cluster barrier; CTA q sums its share of the columns over the
-//           cluster's CTAs in rank order, divides by the summed normaliser and
-//           stores bf16.  No atomics: bit-reproducible.
+//           of lanes reads the K1 part in 16-byte chunks (all of the CTA's keys
+//           in flight at once, issued together with the query chunks) and
+//           reduces with shuffles.
+//  stats    the CTA's (count, mean, M2, max), two passes over shared memory,
+//           pushed into every CTA's inbox; one cluster barrier; every thread
+//           merges the CS records in rank order, so all derive the same bits of
+//           theta and of the score maximum M.
+//  gather   each warp takes its own blocks of 32 keys, lists their selected keys
+//           and, for a batch of them at a time, loads the K2 part and the value
+//           row together: a = <K2[j], q[r:]>, w = exp(s_j - M),
+//           f = w softplus(a), numerator += f V[j], normaliser += w.
+//  reduce   the CTA sums its warps' partials in warp order and pushes column c
+//           to the inbox of CTA c / ceil(d_head / CS); one cluster barrier; each
+//           CTA sums its columns over the cluster in rank order, divides by the
+//           summed normaliser and stores bf16.  No atomics: bit-reproducible.
+// Remote shared memory is only ever written (st.shared::cluster) and only read
+// locally after a barrier; the first remote store waits on a barrier phase that
+// every CTA arrived at on entry, so no CTA writes into one that has not started.
 #include <cstdlib>
 
 #include "spark_device.cuh"
@@ -36,7 +42,8 @@ namespace {
 constexpr int kAThreads = 256;
 constexpr int kAWarps = kAThreads / 32;
 constexpr int kMaxDHead = 256;           // 32 chunks of 16 bytes per key row
-constexpr int kKeyBatch = 8;             // key-steps in flight per lane in the score loop
+constexpr int kKeyBatch = 16;            // key-steps in flight per lane in the score loop
+constexpr int kGather = 8;               // selected keys in flight per warp in the gather
 
 struct AttnParams {
   const uint16_t* q;  // bf16 [n_heads][d_head]
@@ -61,12 +68,19 @@ __device__ __forceinline__ void cluster_sync_a() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ float ld_dsmem(const float* p, unsigned rank) {
+__device__ __forceinline__ void cluster_arrive_relaxed_a() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait_a() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// store v into the same offset of CTA `rank`'s shared memory
+__device__ __forceinline__ void st_dsmem(float* p, unsigned rank, float v) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(p)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ uint4 ldg_ro(const void* p) {
@@ -82,59 +96,57 @@ __device__ __forceinline__ float softplus_f(float a) {
 
 // Shared-memory layout (dynamic part).
 struct ALayout {
-  size_t qs, ss, act_i, act_f, act_w, red, part, stats, misc, total;
-  __host__ __device__ ALayout(int d_head, int kpc) {
+  size_t ss, lists, red, redz, in_stats, in_part, in_z, total;
+  int seg;  // list capacity of one warp: its blocks of 32 keys
+  __host__ __device__ ALayout(int kpc) {
+    const int blocks = (kpc + 31) / 32;
+    seg = (blocks + kAWarps - 1) / kAWarps * 32;
     size_t off = 0;
-    qs = off;
-    off += static_cast<size_t>(kMaxDHead) * 2;
-    ss = off;
+    ss = off;  // the CTA's scores
     off += static_cast<size_t>(kpc) * 4;
-    act_i = off;
-    off += static_cast<size_t>(kpc) * 4;
-    act_f = off;
-    off += static_cast<size_t>(kpc) * 4;
-    act_w = off;
-    off += static_cast<size_t>(kpc) * 4;
-    red = off;  // per-group partial numerators [kAWarps][kMaxDHead]
+    lists = off;  // per-warp lists of selected keys [kAWarps][seg]
+    off += static_cast<size_t>(kAWarps) * seg * 4;
+    red = off;  // per-warp partial numerators [kAWarps][kMaxDHead]
     off += static_cast<size_t>(kAWarps) * kMaxDHead * 4;
-    part = off;  // this CTA's partial numerator, read by the cluster
-    off += static_cast<size_t>(kMaxDHead) * 4;
-    stats = off;  // (count, mean, M2, max, normaliser), read by the cluster
-    off += 32;
-    misc = off;
-    off += 64;
+    redz = off;  // per-warp partial normalisers
+    off += kAWarps * 4;
+    in_stats = off;  // inbox: (count, mean, M2, max) of every CTA of the cluster
+    off += 16 * 4 * 4;
+    in_part = off;  // inbox: [CS][ceil(d_head / CS)] column partials
+    off += (kMaxDHead + 16) * 4;
+    in_z = off;  // inbox: every CTA's normaliser
+    off += 16 * 4;
     total = off;
-    (void)d_head;
   }
 };
 
+// Two CTAs per SM (at most 128 registers a thread): a GPU with fewer than
+// sixteen free SMs in some of its GPCs still holds one 16-CTA cluster per head
+// of an 8-head call resident at once, instead of running the last one as a
+// second wave.
 template <int CS>
-__global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kAThreads, 2) attn_decode_kernel(const AttnParams p) {
   extern __shared__ __align__(128) unsigned char smem[];
+  // every CTA of the cluster has started once this phase completes
+  cluster_arrive_relaxed_a();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned rank = cluster_rank_a();
   const int h = blockIdx.x / CS;
   const int g = h / p.group;
-  const ALayout L(p.d_head, p.kpc);
-  uint16_t* qs = reinterpret_cast<uint16_t*>(smem + L.qs);
+  const ALayout L(p.kpc);
   float* ss = reinterpret_cast<float*>(smem + L.ss);
-  int* act_i = reinterpret_cast<int*>(smem + L.act_i);
-  float* act_f = reinterpret_cast<float*>(smem + L.act_f);
-  float* act_w = reinterpret_cast<float*>(smem + L.act_w);
+  int* list = reinterpret_cast<int*>(smem + L.lists) + warp * L.seg;
   float* red = reinterpret_cast<float*>(smem + L.red);
-  float* part = reinterpret_cast<float*>(smem + L.part);
-  float* stats = reinterpret_cast<float*>(smem + L.stats);
-  float* misc_f = reinterpret_cast<float*>(smem + L.misc);
-  int* misc_i = reinterpret_cast<int*>(smem + L.misc) + 8;
+  float* redz = reinterpret_cast<float*>(smem + L.redz);
+  float* in_stats = reinterpret_cast<float*>(smem + L.in_stats);
+  float* in_part = reinterpret_cast<float*>(smem + L.in_part);
+  float* in_z = reinterpret_cast<float*>(smem + L.in_z);
   const int D = p.d_head;
   const int j0 = static_cast<int>(rank) * p.kpc;
   const int nk = max(0, min(p.kpc, p.n_ctx - j0));
   const uint16_t* Kg = p.K + static_cast<size_t>(g) * p.n_ctx * D;
   const uint16_t* Vg = p.V + static_cast<size_t>(g) * p.n_ctx * D;
-
-  for (int ch = tid; ch < D / 8; ch += kAThreads)
-    *reinterpret_cast<uint4*>(qs + ch * 8) = ldg_ro(p.q + static_cast<size_t>(h) * D + ch * 8);
-  __syncthreads();
+  const uint16_t* qh = p.q + static_cast<size_t>(h) * D;
 
   // ---------------------------------------------------------------- scores
   // a key's K1 part is cpk 16-byte chunks, read by a group of lpk lanes; a warp
@@ -145,7 +157,9 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const AttnPar
   const int kps = 32 / lpk;
   const int cc = lane % lpk, ko = lane / lpk;
   const bool cok = cc < cpk;
-  const uint4 qv = cok ? lds128(qs + cc * 8) : make_uint4(0, 0, 0, 0);
+  const int cpk2 = (D - p.r) / 8;
+  const uint4 qv = cok ? ldg_ro(qh + cc * 8) : make_uint4(0, 0, 0, 0);
+  const uint4 q2 = lane < cpk2 ? ldg_ro(qh + p.r + lane * 8) : make_uint4(0, 0, 0, 0);
   for (int base = warp * kps * kKeyBatch; base < nk; base += kAWarps * kps * kKeyBatch) {
     uint4 kv[kKeyBatch];
 #pragma unroll
@@ -167,6 +181,7 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const AttnPar
       }
   }
   __syncthreads();
+  cluster_wait_a();
 
   // ---------------------------------------------------------------- statistics
   if (warp == 0) {
@@ -184,113 +199,85 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const AttnPar
       const float d = ss[i] - mean;
       m2 = fmaf(d, d, m2);
     }
-    m2 = warp_sum(m2);
-    if (lane == 0) {
-      stats[0] = static_cast<float>(nk);
-      stats[1] = mean;
-      stats[2] = m2;
-      stats[3] = mx;
+    m2 = __shfl_sync(0xffffffffu, warp_sum(m2), 0);
+    if (lane < CS) {
+      float* slot = in_stats + rank * 4;
+      st_dsmem(slot + 0, lane, static_cast<float>(nk));
+      st_dsmem(slot + 1, lane, mean);
+      st_dsmem(slot + 2, lane, m2);
+      st_dsmem(slot + 3, lane, mx);
     }
   }
   cluster_sync_a();
-  if (tid == 0) {
-    // the cluster's records merged in rank order: the same bits in every CTA
-    float n[CS], mu[CS], m2[CS];
-    float N = 0.f, sx = 0.f, mx = -__int_as_float(0x7f800000);
+  // the cluster's records merged by every warp: lane l < CS holds record l and
+  // xor-butterflies combine them; a butterfly adds the same pairs in every lane
+  // (addition commutes), so every thread of every CTA derives the same bits of
+  // theta and of the score maximum M
+  float theta, smax;
+  {
+    const bool own = lane < CS;
+    const float n = own ? in_stats[lane * 4 + 0] : 0.f;
+    const float mu = own ? in_stats[lane * 4 + 1] : 0.f;
+    const float m2 = own ? in_stats[lane * 4 + 2] : 0.f;
+    smax = own ? in_stats[lane * 4 + 3] : -__int_as_float(0x7f800000);
+    float N = n, sx = n * mu;
 #pragma unroll
-    for (int src = 0; src < CS; ++src) {
-      n[src] = ld_dsmem(stats + 0, src);
-      mu[src] = ld_dsmem(stats + 1, src);
-      m2[src] = ld_dsmem(stats + 2, src);
-      mx = fmaxf(mx, ld_dsmem(stats + 3, src));
-    }
-#pragma unroll
-    for (int src = 0; src < CS; ++src) {
-      N += n[src];
-      sx = fmaf(n[src], mu[src], sx);
+    for (int off = 16; off > 0; off >>= 1) {
+      N += __shfl_xor_sync(0xffffffffu, N, off);
+      sx += __shfl_xor_sync(0xffffffffu, sx, off);
+      smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, off));
     }
     const float mean = sx / fmaxf(N, 1.f);
-    float M2 = 0.f;
+    const float d = mu - mean;
+    float M2 = m2 + n * d * d;
 #pragma unroll
-    for (int src = 0; src < CS; ++src) {
-      const float d = mu[src] - mean;
-      M2 += m2[src] + n[src] * d * d;
-    }
-    misc_f[0] = p.select_all ? -__int_as_float(0x7f800000)
-                             : fmaf(sqrtf(fmaxf(M2, 0.f) / fmaxf(N, 1.f)), p.Q, mean);
-    misc_f[1] = mx;
+    for (int off = 16; off > 0; off >>= 1) M2 += __shfl_xor_sync(0xffffffffu, M2, off);
+    theta = p.select_all ? -__int_as_float(0x7f800000) : fmaf(sqrtf(fmaxf(M2, 0.f) / fmaxf(N, 1.f)), p.Q, mean);
   }
-  __syncthreads();
-  const float theta = misc_f[0];
-  const float smax = misc_f[1];
   if (rank == 0 && tid == 0 && p.theta_out != nullptr) p.theta_out[h] = theta;
-  for (int i = tid; i < nk; i += kAThreads) {
-    if (p.s_out != nullptr) p.s_out[static_cast<size_t>(h) * p.n_ctx + j0 + i] = ss[i];
-    if (p.active_out != nullptr) p.active_out[static_cast<size_t>(h) * p.n_ctx + j0 + i] = ss[i] > theta ? 1 : 0;
-  }
+  if (p.s_out != nullptr || p.active_out != nullptr)
+    for (int i = tid; i < nk; i += kAThreads) {
+      if (p.s_out != nullptr) p.s_out[static_cast<size_t>(h) * p.n_ctx + j0 + i] = ss[i];
+      if (p.active_out != nullptr) p.active_out[static_cast<size_t>(h) * p.n_ctx + j0 + i] = ss[i] > theta ? 1 : 0;
+    }
 
   // ---------------------------------------------------------------- gather
-  // the selected keys of this CTA, ascending
-  if (warp == 0) {
-    int cnt = 0;
-    for (int base = 0; base < nk; base += 32) {
-      const int i = base + lane;
-      const bool act = i < nk && ss[i] > theta;
-      const unsigned ball = __ballot_sync(0xffffffffu, act);
-      if (act) act_i[cnt + __popc(ball & ((1u << lane) - 1u))] = i;
-      cnt += __popc(ball);
-    }
-    if (lane == 0) misc_i[0] = cnt;
+  // warp w lists the selected keys of its blocks w, w + 8, ... in ascending order
+  int cnt = 0;
+  for (int b = warp * 32; b < nk; b += kAWarps * 32) {
+    const int i = b + lane;
+    const bool act = i < nk && ss[i] > theta;
+    const unsigned ball = __ballot_sync(0xffffffffu, act);
+    if (act) list[cnt + __popc(ball & ((1u << lane) - 1u))] = i;
+    cnt += __popc(ball);
   }
-  __syncthreads();
-  const int nact = misc_i[0];
-  // f_j = exp(s_j - M) softplus(<K2[j], q[r:]>): one warp per key, four keys'
-  // loads in flight before the arithmetic
-  const int cpk2 = (D - p.r) / 8;
-  constexpr int kKB = 4;
-  const uint4 q2 = lane < cpk2 ? lds128(qs + p.r + lane * 8) : make_uint4(0, 0, 0, 0);
-  for (int jb = warp * kKB; jb < nact; jb += kAWarps * kKB) {
-    uint4 kv[kKB];
-#pragma unroll
-    for (int u = 0; u < kKB; ++u) {
-      const int jj = jb + u;
-      kv[u] = (jj < nact && lane < cpk2)
-                  ? ldg_ro(Kg + static_cast<size_t>(j0 + act_i[jj]) * D + p.r + lane * 8)
-                  : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int u = 0; u < kKB; ++u) {
-      const float a = warp_sum(dot8_bf16(kv[u], q2, 0.f));
-      const int jj = jb + u;
-      if (lane == 0 && jj < nact) {
-        const float w = __expf(ss[act_i[jj]] - smax);
-        act_w[jj] = w;
-        act_f[jj] = w * softplus_f(a);
-      }
-    }
-  }
-  __syncthreads();
-  // partial numerator: warp w sums the keys w, w + 8, ... over column chunk `lane`
+  __syncwarp();
+  // K2 part (lanes < cpk2) and value row (lanes < cpr) of kGather keys in flight
   const int cpr = D / 8;
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  constexpr int kVB = 8;
-  for (int jb = warp; jb < nact; jb += kAWarps * kVB) {
-    uint4 v[kVB];
+  float zw = 0.f;
+  for (int jb = 0; jb < cnt; jb += kGather) {
+    uint4 kv[kGather], vv[kGather];
+    int idx[kGather];
 #pragma unroll
-    for (int u = 0; u < kVB; ++u) {
-      const int jj = jb + u * kAWarps;
-      v[u] = (jj < nact && lane < cpr) ? ldg_ro(Vg + static_cast<size_t>(j0 + act_i[jj]) * D + lane * 8)
-                                       : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < kGather; ++u) {
+      idx[u] = jb + u < cnt ? list[jb + u] : -1;
+      const size_t row = static_cast<size_t>(j0 + max(idx[u], 0)) * D;
+      kv[u] = (idx[u] >= 0 && lane < cpk2) ? ldg_ro(Kg + row + p.r + lane * 8) : make_uint4(0, 0, 0, 0);
+      vv[u] = (idx[u] >= 0 && lane < cpr) ? ldg_ro(Vg + row + lane * 8) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < kVB; ++u) {
-      const int jj = jb + u * kAWarps;
-      if (jj < nact) {
-        const float f = act_f[jj];
-        const float2 v0 = bf16x2_to_float2(v[u].x), v1 = bf16x2_to_float2(v[u].y);
-        const float2 v2 = bf16x2_to_float2(v[u].z), v3 = bf16x2_to_float2(v[u].w);
+    for (int u = 0; u < kGather; ++u) {
+      // every lane scales its value chunk by f: the sum is broadcast from lane 0
+      const float a = __shfl_sync(0xffffffffu, warp_sum(dot8_bf16(kv[u], q2, 0.f)), 0);
+      if (idx[u] >= 0) {
+        const float w = __expf(ss[idx[u]] - smax);
+        const float f = w * softplus_f(a);
+        zw += w;
+        const float2 v0 = bf16x2_to_float2(vv[u].x), v1 = bf16x2_to_float2(vv[u].y);
+        const float2 v2 = bf16x2_to_float2(vv[u].z), v3 = bf16x2_to_float2(vv[u].w);
         acc[0] = fmaf(f, v0.x, acc[0]);
         acc[1] = fmaf(f, v0.y, acc[1]);
         acc[2] = fmaf(f, v1.x, acc[2]);
@@ -305,37 +292,36 @@ __global__ void __launch_bounds__(kAThreads, 1) attn_decode_kernel(const AttnPar
   if (lane < cpr)
 #pragma unroll
     for (int e = 0; e < 8; ++e) red[warp * kMaxDHead + lane * 8 + e] = acc[e];
-  // partial normaliser, fixed order
-  if (warp == 0) {
-    float z = 0.f;
-    for (int jj = lane; jj < nact; jj += 32) z += act_w[jj];
-    z = warp_sum(z);
-    if (lane == 0) stats[4] = z;
-  }
+  if (lane == 0) redz[warp] = zw;
   __syncthreads();
+
+  // ---------------------------------------------------------------- reduce over the cluster
+  // column c goes to CTA c / cw, slot (rank, c % cw); the normaliser to every CTA
+  const int cw = (D + CS - 1) / CS;
   for (int col = tid; col < D; col += kAThreads) {
     float sum = 0.f;
 #pragma unroll
     for (int w = 0; w < kAWarps; ++w) sum += red[w * kMaxDHead + col];
-    part[col] = sum;
+    st_dsmem(in_part + rank * cw + col % cw, static_cast<unsigned>(col / cw), sum);
   }
-
-  // ---------------------------------------------------------------- reduce over the cluster
+  if (tid < CS) {
+    float z = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAWarps; ++w) z += redz[w];
+    st_dsmem(in_z + rank, static_cast<unsigned>(tid), z);
+  }
   cluster_sync_a();
-  const int cw = (D + CS - 1) / CS;
   const int col = static_cast<int>(rank) * cw + tid;
   if (tid < cw && col < D) {
     float num = 0.f, z = 0.f;
 #pragma unroll
     for (int src = 0; src < CS; ++src) {
-      num += ld_dsmem(part + col, static_cast<unsigned>(src));
-      z += ld_dsmem(stats + 4, static_cast<unsigned>(src));
+      num += in_part[src * cw + tid];
+      z += in_z[src];
     }
     const __nv_bfloat16 b = __float2bfloat16_rn(z > 0.f ? num / z : 0.f);
     p.out[static_cast<size_t>(h) * D + col] = *reinterpret_cast<const uint16_t*>(&b);
   }
-  // no CTA leaves while another may still read its shared memory
-  cluster_sync_a();
 }
 
 }  // namespace
@@ -373,7 +359,7 @@ cudaError_t launch_attn_decode(const AttnArgs& a, int num_sms, cudaStream_t stre
   p.s_out = a.s_out;
   p.theta_out = a.theta_out;
   p.active_out = a.active_out;
-  const size_t smem = ALayout(a.d_head, p.kpc).total;
+  const size_t smem = ALayout(p.kpc).total;
   auto kern = cs == 16 ? attn_decode_kernel<16> : attn_decode_kernel<8>;
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

@@ -47,7 +47,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill / stat-topk extra lines")
-    ap.add_argument("--case", default=None, choices=["decode", "prefill", "topk"],
+    ap.add_argument("--case", default=None, choices=["decode", "prefill", "topk", "attention"],
                     help="profiling mode: run only this workload, plain launches (no graph), print per-call time")
     ap.add_argument("--tokens", type=int, default=256, help="--case prefill: tokens per call")
     return ap.parse_args()
@@ -274,7 +274,17 @@ def run_case(args):
     import activation_sparse_transformer_predictor_b200 as spark
     from activation_sparse_transformer_predictor_b200 import synthetic
     dev = torch.device("cuda", 0)
-    if args.case == "topk":
+    if args.case == "attention":
+        import math as _m
+        caches = []
+        for c in range(4):
+            host = synthetic.attention_inputs(8, 4, 4096, 256, layer=c)
+            caches.append({n: t.to(dev) for n, t in host.items()})
+        aout = torch.empty_like(caches[0]["q"])
+        fn = lambda i: spark.attention_decode(caches[i % 4]["q"], caches[i % 4]["K"], caches[i % 4]["V"], 128, 256,
+                                              scale=1.0 / _m.sqrt(256), out=aout)
+        unit = "attention 8/4 heads x 4096 positions"
+    elif args.case == "topk":
         rows, d, k = 8 * 4096, 4096, 256
         x = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
         out = torch.empty_like(x)
