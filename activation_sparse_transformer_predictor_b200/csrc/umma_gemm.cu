@@ -39,8 +39,12 @@ namespace {
 constexpr int BM = 128;
 constexpr int BN = 128;
 constexpr int BK = 64;
-constexpr int kGemmThreads = 192;
-constexpr int kEpiThreads = 128;
+// warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; the rest: epilogue.
+// GEMM 2's gate epilogue (GELU, split, score loads: a chain of dependent
+// latencies per element) runs eight epilogue warps, two per TMEM lane quarter,
+// each on its own half of the tile's columns; the others run four.
+__host__ __device__ constexpr int epi_warps(int epi) { return epi == 2 ? 8 : 4; }
+__host__ __device__ constexpr int gemm_threads(int epi) { return 64 + 32 * epi_warps(epi); }
 constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kBBytes = BN * BK * 2;  // 16 KB
 
@@ -49,13 +53,15 @@ enum Epilogue : int { kEpiPredictor = 1, kEpiGate = 2, kEpiOut = 3 };
 struct GemmParams {
   int M, N, K;
   int tiles_m, tiles_n, split_k, kb_per_split, nkb, units;
-  int nkb0;               // GEMM 2: k-blocks of the first segment (Q1 K1^T); the rest is Q2 K2^T
-  float* X;               // optional predictor scores [M][N] written by GEMM 1 (debug)
+  float* X;               // optional predictor scores [M][N] fp32, row-major (debug copy)
+  float4* Xt;             // predictor scores in 128 x 128 tiles: written by GEMM 1, read by GEMM 2
+  int xt_tiles_n;         // 128-column tiles per 128-row band of Xt
   float2* moments;        // [M][mom_stride] (mean, M2) of each 128-neuron tile
   int mom_stride;         // 128-neuron tiles per row of moments
   const float* theta;     // [M]
-  uint16_t* h_hi;         // [M][N] bf16
-  uint16_t* h_lo;         // [M][N] bf16
+  uint16_t* h_hi;         // bf16, blocked: see h_block()
+  uint16_t* h_lo;         // bf16, blocked like h_hi
+  int h_kb;               // 64-neuron blocks per 128-token band of h_hi / h_lo
   unsigned char* active;  // optional [M][N]
   float* part;            // GEMM 3 split-K partials [split][M][N]
   uint16_t* out;          // GEMM 3 bf16 output [M][N] when split_k == 1
@@ -119,6 +125,12 @@ __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) {
   return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
          (2ull << 61);
 }
+// K-major without swizzle: 8-row x 16-byte core matrices, 128 B each; lbo bytes
+// between the two core matrices of one K 16 step, sbo bytes between 8-row groups.
+__device__ __forceinline__ uint64_t desc_kmajor_none(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
 // N-major: 64 bf16 along N per 128-byte row, one row per K index, 8-row atoms
 // 1024 B apart along K; the two 64-wide N halves of the tile are lbo bytes apart.
 __device__ __forceinline__ uint64_t desc_nmajor_sw128(uint32_t saddr, uint32_t lbo) {
@@ -137,33 +149,71 @@ __device__ __forceinline__ uint16_t f2bf(float f) {
   return *reinterpret_cast<const uint16_t*>(&b);
 }
 
-__device__ __forceinline__ float bf2f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+__device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 b) { return *reinterpret_cast<const uint32_t*>(&b); }
 
+
+// Unit order: GEMMs 1 and 2 walk the token tiles under one neuron tile, so the
+// weight tile (K1 / K2 rows, read once from HBM) is shared by consecutive units
+// while the small token operand stays in L2.  GEMM 3 walks the output columns
+// under one token tile: its A operand (h, T x d_ff, larger than L2 at long
+// prompts) is then read from HBM once, and V (d_ff x d_model) stays in L2.
+template <int EPI>
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int unit, int& tm, int& tn, int& kb0, int& kb1) {
   const int per_split = p.tiles_m * p.tiles_n;
   const int split = unit / per_split;
   const int rem = unit % per_split;
-  tn = rem / p.tiles_m;  // consecutive units share an N tile: B tile reuse in L2
-  tm = rem % p.tiles_m;
+  if (EPI == kEpiOut) {
+    tm = rem / p.tiles_n;
+    tn = rem % p.tiles_n;
+  } else {
+    tn = rem / p.tiles_m;
+    tm = rem % p.tiles_m;
+  }
   kb0 = split * p.kb_per_split;
   kb1 = min(p.nkb, kb0 + p.kb_per_split);
 }
 
-// WIDE (GEMM 1 only): a unit is 128 rows x 256 columns, two 128-column halves
+// Tiled score layout: the 128 x 128 tile (tm, tn) is 64 KB contiguous; inside
+// it, float4 i (columns 4i..4i+3) of row `row` sits at [i][row], so that the 32
+// lanes of an epilogue warp (32 consecutive rows) store or load 512 contiguous
+// bytes per instruction.
+__device__ __forceinline__ float4* xt_tile(const GemmParams& p, int tm, int nb) {
+  return p.Xt + (static_cast<size_t>(tm) * p.xt_tiles_n + nb / BN) * (BN / 4) * BM;
+}
+
+// The gated activations h_hi / h_lo (the A operand of GEMM 3) are stored in
+// blocks of 128 tokens x 64 neurons, 16 KB contiguous each, block (tm, kb) at
+// (tm * h_kb + kb) * 16 KB; inside a block, 16-byte chunk c (neurons 8c..8c+7)
+// of token row r sits at c * 2048 + r * 16.  That is the tensor core's K-major
+// no-swizzle operand layout as it stands, so GEMM 3 fetches a block with one
+// bulk copy, and the 32 lanes of a GEMM 2 epilogue warp (32 consecutive rows)
+// store 512 contiguous bytes per instruction.
+constexpr int kHBlockBytes = BM * BK * 2;  // 16 KB
+__device__ __forceinline__ uint4* h_block(uint16_t* h, const GemmParams& p, int tm, int kb) {
+  return reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(h) +
+                                  (static_cast<size_t>(tm) * p.h_kb + kb) * kHBlockBytes);
+}
+
+// GEMM 2 epilogue: float4 group i of row `row` of the scores [nb, nb + 128), as
+// GEMM 1 stored them (N is a multiple of 16: a group of four is wholly inside)
+__device__ __forceinline__ float4 gate_x(const GemmParams& p, const float4* tile, int row, int nb, int i) {
+  return nb + 4 * i < p.N ? __ldcg(tile + i * BM + row) : make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// WIDE (GEMMs 1 and 2): a unit is 128 rows x 256 columns, two 128-column halves
 // that share the A tile of each stage and own one half of the accumulator each;
 // each k-step issues the same M 128, N 128, K 16 instruction once per half, so
 // every output element sees the instruction sequence of the narrow tile.
 template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(EPI), 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const GemmParams p) {
-  static_assert(!WIDE || (EPI == kEpiPredictor && !B_NMAJOR && !DUAL), "wide units are for GEMM 1");
+  static_assert(!WIDE || (EPI != kEpiOut && !B_NMAJOR && !DUAL), "wide units are for GEMMs 1 and 2");
+  static_assert(!DUAL || EPI == kEpiOut, "two A operands (h_hi, h_lo) are GEMM 3's");
   constexpr int kBTiles = WIDE ? 2 : 1;
   constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes * kBTiles;
-  // GEMM 2 keeps two accumulators per tile (x and a): two segments of k-blocks
-  constexpr bool TWO = EPI == kEpiGate;
-  constexpr int kAccCols = (TWO || WIDE) ? 2 * BN : BN;   // TMEM columns of one tile's accumulators
+  constexpr int kAccCols = WIDE ? 2 * BN : BN;  // TMEM columns of one tile's accumulators
   constexpr int kTmemCols = 2 * kAccCols;       // double buffered
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -185,7 +235,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiThreads);
+      mbar_init(&tempty[a], 32 * epi_warps(EPI));
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -204,7 +254,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.units; unit += gridDim.x) {
       int tm, tn, kb0, kb1;
-      decode_unit(p, unit, tm, tn, kb0, kb1);
+      decode_unit<EPI>(p, unit, tm, tn, kb0, kb1);
+      if (EPI == kEpiGate) {
+        // the gate epilogue reads this unit's score tiles a whole main loop from
+        // now: pull them into L2 (a 64 KB tile is contiguous)
+#pragma unroll
+        for (int h = 0; h < kBTiles; ++h)
+          if ((tn * kBTiles + h) * BN < p.N) prefetch_l2_bulk(xt_tile(p, tm, (tn * kBTiles + h) * BN), BM * BN * 4);
+      }
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, p.wait_limit_ns, ctl, 100) || *abort_flag) {
           *abort_flag = 1;
@@ -214,20 +271,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         unsigned char* sa = smem + stage * kStageBytes;
         mbar_arrive_expect_tx(&full[stage], kStageBytes);
         unsigned char* sb = sa + kABytes * (DUAL ? 2 : 1);
-        if (TWO && kb >= p.nkb0) {
-          tma_load_2d(sa, &tmA2, (kb - p.nkb0) * BK, tm * BM, &full[stage]);
-          tma_load_2d(sb, &tmB2, (kb - p.nkb0) * BK, tn * BN, &full[stage]);
+        if (EPI == kEpiOut) {
+          // h_hi and h_lo blocks: already in the operand layout
+          bulk_g2s(sa, h_block(p.h_hi, p, tm, kb), kHBlockBytes, &full[stage]);
+          bulk_g2s(sa + kABytes, h_block(p.h_lo, p, tm, kb), kHBlockBytes, &full[stage]);
         } else {
           tma_load_2d(sa, &tmA, kb * BK, tm * BM, &full[stage]);
           if (DUAL) tma_load_2d(sa + kABytes, &tmA2, kb * BK, tm * BM, &full[stage]);
-          if (B_NMAJOR) {
-            tma_load_2d(sb, &tmB, tn * BN, kb * BK, &full[stage]);
-            tma_load_2d(sb + kBBytes / 2, &tmB, tn * BN + 64, kb * BK, &full[stage]);
-          } else {
+        }
+        if (B_NMAJOR) {
+          tma_load_2d(sb, &tmB, tn * BN, kb * BK, &full[stage]);
+          tma_load_2d(sb + kBBytes / 2, &tmB, tn * BN + 64, kb * BK, &full[stage]);
+        } else {
 #pragma unroll
-            for (int h = 0; h < kBTiles; ++h)
-              tma_load_2d(sb + h * kBBytes, &tmB, kb * BK, (tn * kBTiles + h) * BN, &full[stage]);
-          }
+          for (int h = 0; h < kBTiles; ++h)
+            tma_load_2d(sb + h * kBBytes, &tmB, kb * BK, (tn * kBTiles + h) * BN, &full[stage]);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -268,17 +326,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     bool ok = true;
     for (int unit = blockIdx.x; ok && unit < p.units; unit += gridDim.x) {
       int tm, tn, kb0, kb1;
-      decode_unit(p, unit, tm, tn, kb0, kb1);
+      decode_unit<EPI>(p, unit, tm, tn, kb0, kb1);
       if (!mbar_wait_bounded(&tempty[acc], (uses[acc] & 1u) ^ 1u, p.wait_limit_ns, ctl, 110) || *abort_flag) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t d_base = tmem_base + static_cast<uint32_t>(acc * kAccCols);
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * kAccCols);
       for (int kb = kb0; kb < kb1; ++kb) {
-        const bool seg1 = TWO && kb >= p.nkb0;
-        const uint32_t d_tmem = d_base + (seg1 ? static_cast<uint32_t>(BN) : 0u);
-        const bool first = kb == kb0 || (TWO && kb == p.nkb0);
+        const bool first = kb == kb0;
         if (!mbar_wait_bounded(&full[stage], ph, p.wait_limit_ns, ctl, 111) || *abort_flag) {
           *abort_flag = 1;
           ok = false;
@@ -291,8 +347,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int k = 0; k < BK / 16; ++k) {
           const uint64_t bdesc = B_NMAJOR ? desc_nmajor_sw128(sb + k * 16 * 128, kBBytes / 2)
                                           : desc_kmajor_sw128(sb + k * 32);
-          umma_bf16(d_tmem, desc_kmajor_sw128(sa + k * 32), bdesc, idesc, (!first || k > 0) ? 1u : 0u);
-          if (DUAL) umma_bf16(d_tmem, desc_kmajor_sw128(sa + kABytes + k * 32), bdesc, idesc, 1u);
+          // GEMM 3's A: chunks 2k and 2k + 1 of the h block (2048 B apart), 8-row groups 128 B apart
+          const uint64_t adesc = EPI == kEpiOut ? desc_kmajor_none(sa + k * 4096, 2048, 128)
+                                                : desc_kmajor_sw128(sa + k * 32);
+          umma_bf16(d_tmem, adesc, bdesc, idesc, (!first || k > 0) ? 1u : 0u);
+          if (DUAL) umma_bf16(d_tmem, desc_kmajor_none(sa + kABytes + k * 4096, 2048, 128), bdesc, idesc, 1u);
           if (WIDE)
             umma_bf16(d_tmem + static_cast<uint32_t>(BN), desc_kmajor_sw128(sa + k * 32),
                       desc_kmajor_sw128(sb + kBBytes + k * 32), idesc, (!first || k > 0) ? 1u : 0u);
@@ -312,20 +371,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes [32 quarter, 32 quarter + 32)
     const int row = quarter * 32 + lane;
+    const int colgrp = (warp - 2) >> 2;  // gate epilogue: which half of the columns
     uint32_t uses[2] = {0u, 0u};
     int acc = 0;
     for (int unit = blockIdx.x; unit < p.units; unit += gridDim.x) {
       int tm, tn, kb0, kb1;
-      decode_unit(p, unit, tm, tn, kb0, kb1);
+      decode_unit<EPI>(p, unit, tm, tn, kb0, kb1);
+      const int m = tm * BM + row;
+      const int n_base = tn * BN * kBTiles;
+      const bool row_ok = m < p.M;
+      // GEMM 2: this warp's columns of the tile (a wide unit's half, or half of a
+      // narrow unit) and this row's scores there, stored by GEMM 1, loaded while
+      // the accumulator is still being formed
+      constexpr int kGateCols = WIDE ? BN : BN / 2;
+      const int gcol = colgrp * kGateCols;                // first column within the unit
+      const int gtile_nb = n_base + (WIDE ? gcol : 0);    // first column of its score tile
+      const int gx0 = WIDE ? 0 : gcol / 4;                // its first float4 group in that tile
+      float4 xr[EPI == kEpiGate ? kGateCols / 4 : 1];
+      if (EPI == kEpiGate) {
+        const float4* t0 = xt_tile(p, tm, gtile_nb);
+#pragma unroll
+        for (int i = 0; i < kGateCols / 4; ++i) xr[i] = gate_x(p, t0, row, gtile_nb, gx0 + i);
+      }
       if (!mbar_wait_bounded(&tfull[acc], uses[acc] & 1u, p.wait_limit_ns, ctl, 120) || *abort_flag) {
         *abort_flag = 1;
         break;
       }
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
-      const int m = tm * BM + row;
-      const int n_base = tn * BN * kBTiles;
-      const bool row_ok = m < p.M;
       float v[16];
       if (EPI == kEpiPredictor) {
         float* xrow = p.X + static_cast<size_t>(m) * p.N;
@@ -334,6 +407,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           // one 128-column half: moments about its mean (two passes over TMEM)
           const int nb = n_base + h * BN;
           const uint32_t ta = taddr + static_cast<uint32_t>(h * BN);
+          float4* xt = xt_tile(p, tm, nb);
           float sum = 0.f;
           int cnt = 0;
 #pragma unroll 1
@@ -346,6 +420,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 sum += v[j];
                 ++cnt;
               }
+            if (row_ok && n < p.N) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                xt[(c / 4 + q4) * BM + row] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            }
             if (row_ok && p.X != nullptr) {
               if (n + 16 <= p.N) {
                 float4* d = reinterpret_cast<float4*>(xrow + n);
@@ -376,49 +455,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
       } else if (EPI == kEpiGate) {
         const float th = row_ok ? p.theta[m] : 0.f;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          float x[16];
-          tmem_ld16(taddr + c, x);         // recomputed scores
-          tmem_ld16(taddr + BN + c, v);    // a = K2^T q[r:]
-          const int n = n_base + c;
-          if (!row_ok) continue;
-          uint32_t hi[8], lo[8];
-          uint32_t act[4] = {0u, 0u, 0u, 0u};
+        {
+          const int nb = n_base + gcol;
+          const uint32_t ta = taddr + static_cast<uint32_t>(gcol);
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            float h2[2];
+          for (int c = 0; c < kGateCols; c += 16) {
+            tmem_ld16(ta + c, v);  // a = K2^T q[r:]
+            const int n = nb + c;
+            const float x[16] = {xr[c / 4].x,     xr[c / 4].y,     xr[c / 4].z,     xr[c / 4].w,
+                                 xr[c / 4 + 1].x, xr[c / 4 + 1].y, xr[c / 4 + 1].z, xr[c / 4 + 1].w,
+                                 xr[c / 4 + 2].x, xr[c / 4 + 2].y, xr[c / 4 + 2].z, xr[c / 4 + 2].w,
+                                 xr[c / 4 + 3].x, xr[c / 4 + 3].y, xr[c / 4 + 3].z, xr[c / 4 + 3].w};
+            // every row of the block is stored (rows >= M only ever reach output
+            // rows >= M); neurons in [N, next multiple of 64) are stored as zeros,
+            // since GEMM 3 multiplies them with the zero rows TMA fills in for V
+            if (n >= (p.N + BK - 1) / BK * BK) continue;
+            const bool col_ok = n < p.N;
+            uint32_t hi[8], lo[8];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float s = x[j + u] - th;
-              const bool a = s > 0.f && n + j + u < p.N;
-              h2[u] = a ? gelu_tanh(s) * v[j + u] : 0.f;
-              if (a) act[(j + u) >> 2] |= 1u << (8 * ((j + u) & 3));
-            }
-            const uint16_t hb0 = f2bf(h2[0]), hb1 = f2bf(h2[1]);
-            const uint16_t lb0 = f2bf(h2[0] - bf2f(hb0)), lb1 = f2bf(h2[1] - bf2f(hb1));
-            hi[j >> 1] = static_cast<uint32_t>(hb0) | (static_cast<uint32_t>(hb1) << 16);
-            lo[j >> 1] = static_cast<uint32_t>(lb0) | (static_cast<uint32_t>(lb1) << 16);
-          }
-          const size_t off = static_cast<size_t>(m) * p.N + n;
-          if (n + 16 <= p.N) {
-            uint4* dh = reinterpret_cast<uint4*>(p.h_hi + off);
-            uint4* dl = reinterpret_cast<uint4*>(p.h_lo + off);
-            dh[0] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            dh[1] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
-            dl[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            dl[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
-            if (p.active != nullptr)
+            for (int j = 0; j < 16; j += 2) {
+              float h2[2];
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                p.active[off + j] = static_cast<unsigned char>((act[j >> 2] >> (8 * (j & 3))) & 1u);
-          } else {
-            for (int j = 0; j < 16; ++j)
-              if (n + j < p.N) {
-                p.h_hi[off + j] = static_cast<uint16_t>(hi[j >> 1] >> (16 * (j & 1)));
-                p.h_lo[off + j] = static_cast<uint16_t>(lo[j >> 1] >> (16 * (j & 1)));
-                if (p.active != nullptr) p.active[off + j] = static_cast<unsigned char>((act[j >> 2] >> (8 * (j & 3))) & 1u);
+              for (int u = 0; u < 2; ++u) {
+                const float sft = x[j + u] - th;
+                h2[u] = col_ok && sft > 0.f ? gelu_tanh(sft) * v[j + u] : 0.f;
               }
+              // h = h_hi + h_lo: round to bf16, then round the remainder (pairs packed
+              // by one conversion each; element j in the low half)
+              hi[j >> 1] = bf162_bits(__floats2bfloat162_rn(h2[0], h2[1]));
+              const float2 hf = bf16x2_to_float2(hi[j >> 1]);
+              lo[j >> 1] = bf162_bits(__floats2bfloat162_rn(h2[0] - hf.x, h2[1] - hf.y));
+            }
+            // N is a multiple of 16: a 16-column group is wholly inside or outside
+            const int c8 = (n % BK) / 8;  // first of this group's two 16-byte chunks
+            uint4* dh = h_block(p.h_hi, p, tm, n / BK);
+            uint4* dl = h_block(p.h_lo, p, tm, n / BK);
+            dh[c8 * BM + row] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            dh[(c8 + 1) * BM + row] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+            dl[c8 * BM + row] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            dl[(c8 + 1) * BM + row] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+            if (p.active != nullptr && row_ok && col_ok) {
+              const size_t off = static_cast<size_t>(m) * p.N + n;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) p.active[off + j] = x[j] - th > 0.f ? 1 : 0;
+            }
           }
         }
       } else {  // kEpiOut
@@ -573,7 +653,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUten
     set_dev = dev;
   }
   const int grid = p.units < num_sms ? p.units : num_sms;
-  kern<<<grid, kGemmThreads, smem, stream>>>(a, a2, b, b2, p);
+  kern<<<grid, gemm_threads(EPI), smem, stream>>>(a, a2, b, b2, p);
   return cudaGetLastError();
 }
 
@@ -586,7 +666,8 @@ size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms) {
   size_t b = align256(sizeof(DeviceControl));
   b += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));            // moments
   b += align256(static_cast<size_t>(T) * 4);                                   // theta
-  b += 2 * align256(static_cast<size_t>(T) * d_ff * 2);                        // h_hi, h_lo
+  b += 2 * static_cast<size_t>((T + BM - 1) / BM) * ((d_ff + BK - 1) / BK) * BM * BK * 2;  // h_hi, h_lo
+  b += static_cast<size_t>((T + BM - 1) / BM) * tiles_n * BM * BN * 4;         // tiled scores
   const int splits = prefill_splitk(T, d_model, d_ff, num_sms);
   if (splits > 1) b += align256(static_cast<size_t>(splits) * T * d_model * 4);  // partials
   return b;
@@ -609,33 +690,38 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   off += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));
   float* theta = reinterpret_cast<float*>(ws + off);
   off += align256(static_cast<size_t>(T) * 4);
+  const int h_kb = (d_ff + BK - 1) / BK;
+  const size_t h_bytes = static_cast<size_t>((T + BM - 1) / BM) * h_kb * BM * BK * 2;
   uint16_t* h_hi = reinterpret_cast<uint16_t*>(ws + off);
-  off += align256(static_cast<size_t>(T) * d_ff * 2);
+  off += h_bytes;
   uint16_t* h_lo = reinterpret_cast<uint16_t*>(ws + off);
-  off += align256(static_cast<size_t>(T) * d_ff * 2);
+  off += h_bytes;
+  float4* Xt = reinterpret_cast<float4*>(ws + off);
+  off += static_cast<size_t>((T + BM - 1) / BM) * tiles_n * BM * BN * 4;
   const int splits = prefill_splitk(T, d_model, d_ff, num_sms);
   float* part = splits > 1 ? reinterpret_cast<float*>(ws + off) : nullptr;
 
   const uint16_t* q = static_cast<const uint16_t*>(a.q);
-  CUtensorMap tq1, tq2, tk1, tk2, th, tl, tv;
+  CUtensorMap tq1, tq2, tk1, tk2, tv;
   const uint64_t qrow = static_cast<uint64_t>(d_model) * 2;
   if (!make_tmap(&tq1, q, r, T, qrow, BK, BM) || !make_tmap(&tq2, q + r, d2, T, qrow, BK, BM) ||
       !make_tmap(&tk1, a.K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, BN) ||
       !make_tmap(&tk2, a.K2, d2, d_ff, static_cast<uint64_t>(d2) * 2, BK, BN) ||
-      !make_tmap(&th, h_hi, d_ff, T, static_cast<uint64_t>(d_ff) * 2, BK, BM) ||
-      !make_tmap(&tl, h_lo, d_ff, T, static_cast<uint64_t>(d_ff) * 2, BK, BM) ||
       !make_tmap(&tv, a.V, d_model, d_ff, static_cast<uint64_t>(d_model) * 2, 64, BK))
     return cudaErrorInvalidValue;
 
   GemmParams g{};
   g.ctl = reinterpret_cast<DeviceControl*>(ws);
   g.wait_limit_ns = a.wait_limit_ns;
-  g.X = a.x_out;  // scores leave the chip only for the debug entry point
+  g.X = a.x_out;  // row-major copy for the debug entry point only
+  g.Xt = Xt;      // GEMM 1 stores the scores once, tiled; GEMM 2's gate reads them back
+  g.xt_tiles_n = tiles_n;
   g.moments = moments;
   g.mom_stride = tiles_n;
   g.theta = theta;
   g.h_hi = h_hi;
   g.h_lo = h_lo;
+  g.h_kb = h_kb;
   g.active = a.active_out;
   g.part = part;
   g.out = static_cast<uint16_t*>(a.out);
@@ -664,15 +750,20 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   if (e != cudaSuccess) return e;
   theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, tiles_n, a.Q, theta, a.theta_out);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // GEMM 2: X = Q1 K1^T again and A = Q2 K2^T, gate and split (narrow units)
-  g.tiles_n = tiles_n;
-  g.units = g.tiles_m * g.tiles_n;
-  g.K = d_model;
-  g.nkb0 = (r + BK - 1) / BK;
-  g.nkb = g.nkb0 + (d2 + BK - 1) / BK;
+  // GEMM 2: A = Q2 K2^T; the gate h = GELU(max(x - theta, 0)) a with x as GEMM 1
+  // stored it, split into h_hi + h_lo.  Wide units under the same rule as GEMM 1.
+  g.K = d2;
+  g.nkb = (d2 + BK - 1) / BK;
   g.kb_per_split = g.nkb;
-  g.X = nullptr;
-  e = launch_gemm<kEpiGate, false, false, 6>(tq1, tq2, tk1, tk2, g, num_sms, stream);
+  if (wide_units >= num_sms) {
+    g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
+    g.units = wide_units;
+    e = launch_gemm<kEpiGate, false, false, 4, true>(tq2, tq2, tk2, tk2, g, num_sms, stream);
+  } else {
+    g.tiles_n = tiles_n;
+    g.units = g.tiles_m * g.tiles_n;
+    e = launch_gemm<kEpiGate, false, false, 6>(tq2, tq2, tk2, tk2, g, num_sms, stream);
+  }
   if (e != cudaSuccess) return e;
   // GEMM 3: out = H_hi V + H_lo V
   g.N = d_model;
@@ -682,7 +773,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   g.split_k = splits;
   g.kb_per_split = (g.nkb + splits - 1) / splits;
   g.units = g.tiles_m * g.tiles_n * splits;
-  e = launch_gemm<kEpiOut, true, true, 4>(th, tl, tv, tv, g, num_sms, stream);
+  // GEMM 3 takes h_hi / h_lo by bulk copies of whole blocks: no tensor maps for A
+  e = launch_gemm<kEpiOut, true, true, 4>(tv, tv, tv, tv, g, num_sms, stream);
   if (e != cudaSuccess) return e;
   if (splits > 1) {
     const size_t n4 = static_cast<size_t>(T) * d_model / 4;

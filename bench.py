@@ -465,7 +465,7 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
 
         ms, n = time_graph([pre] * 4, reps, args.warmup, world)
         ms = max_over_ranks(ms, world)
-        flops = 2.0 * T * D_FF * (R + D_MODEL + 2 * D_MODEL)  # executed: predictor + gate (x again, a) + 2-part output
+        flops = 2.0 * T * D_FF * (R + (D_MODEL - R) + 2 * D_MODEL)  # executed: predictor + gate (a) + 2-part output
         res[f"prefill_T{T}"] = {"tokens_per_s": T * 1e3 / ms * world, "ms_per_call": ms,
                                 "executed_tflops": flops / (ms * 1e-3) / 1e12,
                                 "note": "one layer; whole call, all five kernels; the masked products run as "
