@@ -138,9 +138,9 @@ __device__ __forceinline__ uint64_t desc_nmajor_sw128(uint32_t saddr, uint32_t l
          (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// kind::f16 instruction descriptor: bf16 A and B, fp32 D, M = 128, N = BN.
-__host__ __device__ constexpr uint32_t make_idesc(bool b_nmajor) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_nmajor ? 1u : 0u) << 16) | (static_cast<uint32_t>(BN >> 3) << 17) |
+// kind::f16 instruction descriptor: bf16 A and B, fp32 D, M = 128, N = n.
+__host__ __device__ constexpr uint32_t make_idesc(bool b_nmajor, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_nmajor ? 1u : 0u) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(BM >> 4) << 24);
 }
 
@@ -200,10 +200,9 @@ __device__ __forceinline__ float4 gate_x(const GemmParams& p, const float4* tile
   return nb + 4 * i < p.N ? __ldcg(tile + i * BM + row) : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// WIDE (GEMMs 1 and 2): a unit is 128 rows x 256 columns, two 128-column halves
-// that share the A tile of each stage and own one half of the accumulator each;
-// each k-step issues the same M 128, N 128, K 16 instruction once per half, so
-// every output element sees the instruction sequence of the narrow tile.
+// WIDE (GEMMs 1 and 2): a unit is 128 rows x 256 columns: each stage holds one
+// A tile and two adjacent 128-row B tiles, and each K 16 step is one M 128 x
+// N 256 instruction into 256 TMEM columns.
 template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false>
 __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
@@ -318,7 +317,9 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     }
   } else if (warp == 1 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc = make_idesc(B_NMAJOR);
+    // a wide unit is one M 128 x N 256 instruction per K 16 step: its two B tiles
+    // are adjacent in shared memory, 8-row atoms 1024 B apart throughout
+    constexpr uint32_t idesc = make_idesc(B_NMAJOR, WIDE ? 2 * BN : BN);
     int stage = 0;
     uint32_t ph = 0;
     uint32_t uses[2] = {0u, 0u};
@@ -352,9 +353,6 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                                                 : desc_kmajor_sw128(sa + k * 32);
           umma_bf16(d_tmem, adesc, bdesc, idesc, (!first || k > 0) ? 1u : 0u);
           if (DUAL) umma_bf16(d_tmem, desc_kmajor_none(sa + kABytes + k * 4096, 2048, 128), bdesc, idesc, 1u);
-          if (WIDE)
-            umma_bf16(d_tmem + static_cast<uint32_t>(BN), desc_kmajor_sw128(sa + k * 32),
-                      desc_kmajor_sw128(sb + kBBytes + k * 32), idesc, (!first || k > 0) ? 1u : 0u);
         }
         umma_commit(&empty[stage]);
         if (++stage == STAGES) {
