@@ -8,8 +8,10 @@ library's C ABI.  The step cycles over 16 copies of the layer's weights
 (1.36 GB, far above the 126 MB L2), so every step reads its weights from HBM.
 
 Also reported in the same JSON line (key "also"): the batched prefill at
-T = 256 tokens, the standalone statistical top-k on 32768 x 4096 fp32 score
-rows (k = 256), both timed the same way.
+T = 16, 64, 256, 1024 and 4096 tokens, the decode variants, the 26-layer
+decode stack, Spark Attention for one decoding position and the standalone
+statistical top-k on 32768 x 4096 fp32 score rows (k = 256), all timed the
+same way.
 
 ``--impl reference`` times the fp64 CPU oracle (the only reference this method
 has: the pages publish no code) on the host cores, on the same workload.
@@ -449,10 +451,11 @@ def main():
 def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
     from activation_sparse_transformer_predictor_b200 import _binding
     L = _binding.lib()
+    bf16_tflops = peaks()[1]  # burst: each prefill call is timed by itself
     res = {}
     # batched prefill, T = 256 and T = 4096 (one layer; whole-call throughput: predictor GEMM, theta,
     # gate GEMM, output GEMM and split-K reduce)
-    for T, reps in ((256, 40), (4096, 8)):
+    for T, reps in ((16, 80), (64, 80), (256, 40), (1024, 16), (4096, 8)):
         q = synthetic.tokens(T, D_MODEL, layer=1).to(dev)
         out = torch.empty_like(q)
 
@@ -466,8 +469,14 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
         ms, n = time_graph([pre] * 4, reps, args.warmup, world)
         ms = max_over_ranks(ms, world)
         flops = 2.0 * T * D_FF * (R + (D_MODEL - R) + 2 * D_MODEL)  # executed: predictor + gate (a) + 2-part output
+        # algorithmic bytes: K1 once, the expected union of the tokens' active K2 / V rows, q and out
+        union = D_FF * (1.0 - (1.0 - K / D_FF) ** T)
+        abytes = D_FF * R * 2 + union * ((D_MODEL - R) + D_MODEL) * 2 + 2 * T * D_MODEL * 2
         res[f"prefill_T{T}"] = {"tokens_per_s": T * 1e3 / ms * world, "ms_per_call": ms,
                                 "executed_tflops": flops / (ms * 1e-3) / 1e12,
+                                "frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / bf16_tflops,
+                                "algorithmic_bytes": abytes,
+                                "frac_of_hbm_peak": abytes / (ms * 1e-3) / 1e9 / hbm_gbs,
                                 "note": "one layer; whole call, all five kernels; the masked products run as "
                                         "dense 128-token tiles (the union of per-token active sets covers "
                                         "~every neuron); per-kernel live spans are in the prefill profile"}
