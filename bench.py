@@ -151,7 +151,9 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU (RANK / WORLD_SIZE / LOCAL_RANK / MASTER_* from the launcher); every rank
+    runs an independent replica and the group only carries the barrier and the max over ranks."""
     import torch
     if n_gpus <= 1 or "RANK" not in os.environ:
         return 0, 1, 0
@@ -159,28 +161,39 @@ def dist_setup(n_gpus):
     import torch.distributed as dist
     rank, world = int(os.environ["RANK"]), int(os.environ["WORLD_SIZE"])
     local = int(os.environ.get("LOCAL_RANK", rank))
-    torch.cuda.set_device(local)
-    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    else:
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return rank, world, local
 
 
-def barrier_sync(world):
+def barrier_sync(world, cuda=True):
     import torch
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-        torch.cuda.synchronize()
+        if cuda:
+            torch.cuda.synchronize()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device="cuda") -> float:
     if world <= 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_call: float, ms_per_call_max: float, world: int) -> float:
+    """Units per second of the whole job: every rank processes units_per_call per call, and the
+    slowest rank's time per call (the max over ranks) paces them all."""
+    return units_per_call * world * 1e3 / ms_per_call_max
 
 
 def time_graph(fn_list, steps, warmup, world):
@@ -374,7 +387,7 @@ def main():
     ms_exch = max_over_ranks(ms_exch, world)
     del os.environ["SPARK_DECODE_IMPL"]
     assert spark.query_status() == 0
-    tok_s = 1e3 / ms_step * world
+    tok_s = whole_job_rate(1, ms_step, world)
     achieved_gbs = bytes_per_token / (ms_step * 1e-3) / 1e9
 
     # ---------------- end to end through the public API: pinned host q in, host out back
@@ -401,11 +414,11 @@ def main():
 
     also = {
         "decode_T1_without_weight_overlap": {
-            "tokens_per_s": 1e3 / ms_plain * world, "us_per_call": ms_plain * 1e3,
+            "tokens_per_s": whole_job_rate(1, ms_plain, world), "us_per_call": ms_plain * 1e3,
             "frac_of_hbm_peak": bytes_per_token / (ms_plain * 1e-3) / 1e9 / hbm_gbs,
             "note": "score kernel launched after the previous call completes"},
         "decode_T1_exchange_kernel": {
-            "tokens_per_s": 1e3 / ms_exch * world, "us_per_call": ms_exch * 1e3,
+            "tokens_per_s": whole_job_rate(1, ms_exch, world), "us_per_call": ms_exch * 1e3,
             "frac_of_hbm_peak": bytes_per_token / (ms_exch * 1e-3) / 1e9 / hbm_gbs,
             "note": "the alternative one-launch kernel (cooperative, speculative K2 rows, one grid exchange)"},
     }
@@ -435,7 +448,7 @@ def main():
                          "duration": "graph replay time per step (three kernels, gaps included)",
                          "algorithmic_bytes_per_launch": bytes_per_token},
             "cpu_baseline": cpu,
-            "e2e": {"value": 1e3 / e2e_ms * world, "unit": "tokens/s", "h2d_bytes_per_step": D_MODEL * 2,
+            "e2e": {"value": whole_job_rate(1, e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": D_MODEL * 2,
                     "d2h_bytes_per_step": D_MODEL * 2,
                     "path": "public Python API per step: pinned q H2D copy, ffn_forward, out D2H copy"},
             "gpu_launches": 2 * n_timed,
@@ -472,7 +485,7 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
         # algorithmic bytes: K1 once, the expected union of the tokens' active K2 / V rows, q and out
         union = D_FF * (1.0 - (1.0 - K / D_FF) ** T)
         abytes = D_FF * R * 2 + union * ((D_MODEL - R) + D_MODEL) * 2 + 2 * T * D_MODEL * 2
-        res[f"prefill_T{T}"] = {"tokens_per_s": T * 1e3 / ms * world, "ms_per_call": ms,
+        res[f"prefill_T{T}"] = {"tokens_per_s": whole_job_rate(T, ms, world), "ms_per_call": ms,
                                 "executed_tflops": flops / (ms * 1e-3) / 1e12,
                                 "frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / bf16_tflops,
                                 "algorithmic_bytes": abytes,
@@ -502,7 +515,7 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
     ms, n = time_graph([stack] * 2, 20, args.warmup, world)
     ms = max_over_ranks(ms, world)
     stack_bytes = n_layers * (D_FF * R * 2 + 737 * (D_MODEL - R + D_MODEL) * 2 + 2 * D_MODEL * 2)
-    res["stack_26_layers_T1"] = {"tokens_per_s": 1e3 / ms * world, "us_per_token": ms * 1e3,
+    res["stack_26_layers_T1"] = {"tokens_per_s": whole_job_rate(1, ms, world), "us_per_token": ms * 1e3,
                                  "us_per_layer": ms * 1e3 / n_layers,
                                  "achieved_GBs": stack_bytes / (ms * 1e-3) / 1e9,
                                  "frac_of_hbm_peak": stack_bytes / (ms * 1e-3) / 1e9 / hbm_gbs,
@@ -534,7 +547,7 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
     ms = max_over_ranks(ms, world)
     abytes = KV * NC * RA * 2 + H * KA * ((DH - RA) + DH) * 2 + 2 * H * DH * 2
     res["spark_attention_decode_8x4096"] = {
-        "calls_per_s": 1e3 / ms * world, "us_per_call": ms * 1e3, "achieved_GBs": abytes / (ms * 1e-3) / 1e9,
+        "calls_per_s": whole_job_rate(1, ms, world), "us_per_call": ms * 1e3, "achieved_GBs": abytes / (ms * 1e-3) / 1e9,
         "frac_of_hbm_peak": abytes / (ms * 1e-3) / 1e9 / hbm_gbs, "algorithmic_bytes_per_call": abytes,
         "note": "one launch, one 16-CTA cluster per query head; bytes = predictor parts of all cached keys + "
                 "K2 parts and value rows of ~256 selected keys per head + q/out; 16 caches (75 MB) cycled"}
@@ -552,7 +565,7 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
     ms, n = time_graph([tk] * 2, 20, args.warmup, world)
     ms = max_over_ranks(ms, world)
     gbs = rows * d * 8 / (ms * 1e-3) / 1e9
-    res["stat_topk_32768x4096"] = {"rows_per_s": rows * 1e3 / ms * world, "ms_per_call": ms, "achieved_GBs": gbs,
+    res["stat_topk_32768x4096"] = {"rows_per_s": whole_job_rate(rows, ms, world), "ms_per_call": ms, "achieved_GBs": gbs,
                                    "frac_of_hbm_peak": gbs / hbm_gbs,
                                    "traffic": profile_traffic("stat_topk_32768x4096.txt", TOPK_SOURCES),
                                    "note": "512 MiB read + 512 MiB written per call (> L2)"}
