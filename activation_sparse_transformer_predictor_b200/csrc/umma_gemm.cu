@@ -41,9 +41,9 @@ constexpr int BN = 128;
 constexpr int BK = 64;
 // warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; the rest: epilogue.
 // GEMM 2's gate epilogue (GELU, split, score loads: a chain of dependent
-// latencies per element) runs eight epilogue warps, two per TMEM lane quarter,
-// each on its own half of the tile's columns; the others run four.
-__host__ __device__ constexpr int epi_warps(int epi) { return epi == 2 ? 8 : 4; }
+// latencies per element) runs sixteen epilogue warps, four per TMEM lane
+// quarter, each on its own quarter of the unit's columns; the others run four.
+__host__ __device__ constexpr int epi_warps(int epi) { return epi == 2 ? 16 : 4; }
 __host__ __device__ constexpr int gemm_threads(int epi) { return 64 + 32 * epi_warps(epi); }
 constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kBBytes = BN * BK * 2;  // 16 KB
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes [32 quarter, 32 quarter + 32)
     const int row = quarter * 32 + lane;
-    const int colgrp = (warp - 2) >> 2;  // gate epilogue: which half of the columns
+    const int colgrp = (warp - 2) >> 2;  // gate epilogue: which quarter of the columns
     uint32_t uses[2] = {0u, 0u};
     int acc = 0;
     for (int unit = blockIdx.x; unit < p.units; unit += gridDim.x) {
@@ -381,10 +381,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       // GEMM 2: this warp's columns of the tile (a wide unit's half, or half of a
       // narrow unit) and this row's scores there, stored by GEMM 1, loaded while
       // the accumulator is still being formed
-      constexpr int kGateCols = WIDE ? BN : BN / 2;
+      constexpr int kGateCols = (WIDE ? 2 * BN : BN) / (epi_warps(kEpiGate) / 4);
       const int gcol = colgrp * kGateCols;                // first column within the unit
-      const int gtile_nb = n_base + (WIDE ? gcol : 0);    // first column of its score tile
-      const int gx0 = WIDE ? 0 : gcol / 4;                // its first float4 group in that tile
+      const int gtile_nb = n_base + gcol / BN * BN;       // first column of its score tile
+      const int gx0 = gcol % BN / 4;                      // its first float4 group in that tile
       float4 xr[EPI == kEpiGate ? kGateCols / 4 : 1];
       if (EPI == kEpiGate) {
         const float4* t0 = xt_tile(p, tm, gtile_nb);
