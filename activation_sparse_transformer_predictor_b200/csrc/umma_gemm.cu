@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const GemmParams p) {
-  static_assert(!WIDE || (EPI != kEpiOut && !B_NMAJOR && !DUAL), "wide units are for GEMMs 1 and 2");
+  static_assert(!WIDE || B_NMAJOR == (EPI == kEpiOut), "wide GEMM 3 takes V N-major; GEMMs 1 and 2 K-major");
   static_assert(!DUAL || EPI == kEpiOut, "two A operands (h_hi, h_lo) are GEMM 3's");
   constexpr int kBTiles = WIDE ? 2 : 1;
   constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes * kBTiles;
@@ -279,8 +279,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           if (DUAL) tma_load_2d(sa + kABytes, &tmA2, kb * BK, tm * BM, &full[stage]);
         }
         if (B_NMAJOR) {
-          tma_load_2d(sb, &tmB, tn * BN, kb * BK, &full[stage]);
-          tma_load_2d(sb + kBBytes / 2, &tmB, tn * BN + 64, kb * BK, &full[stage]);
+          // V rows kb*64.. as 64-column boxes, 8 KB apart (two per 128 columns)
+#pragma unroll
+          for (int h = 0; h < 2 * kBTiles; ++h)
+            tma_load_2d(sb + h * (kBBytes / 2), &tmB, tn * BN * kBTiles + h * 64, kb * BK, &full[stage]);
         } else {
 #pragma unroll
           for (int h = 0; h < kBTiles; ++h)
@@ -502,7 +504,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       } else {  // kEpiOut
         const int split = unit / (p.tiles_m * p.tiles_n);
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
+        for (int c = 0; c < BN * kBTiles; c += 16) {
           tmem_ld16(taddr + c, v);
           const int n = n_base + c;
           if (!row_ok) continue;
@@ -671,8 +673,18 @@ size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms) {
   return b;
 }
 
+// GEMM 3 runs 128 x 256 units (one N 256 instruction per K 16 step, both A
+// halves on each V tile) once there are about a third as many of them as SMs
+// (measured at the Gemma shape: better from T = 1024 on, worse at T <= 256,
+// where the wide units need twice the split-K partials); below that the narrow
+// 128 x 128 units.
+bool prefill_gemm3_wide(int T, int d_model, int num_sms) {
+  return ((T + BM - 1) / BM) * ((d_model + 2 * BN - 1) / (2 * BN)) * 3 >= num_sms;
+}
+
 int prefill_splitk(int T, int d_model, int d_ff, int num_sms) {
-  const int tiles = ((T + BM - 1) / BM) * ((d_model + BN - 1) / BN);
+  const int wn = prefill_gemm3_wide(T, d_model, num_sms) ? 2 * BN : BN;
+  const int tiles = ((T + BM - 1) / BM) * ((d_model + wn - 1) / wn);
   const int nkb = (d_ff + BK - 1) / BK;
   int s = 1;
   while (tiles * s * 2 <= num_sms && s * 2 <= nkb / 4) s *= 2;
@@ -766,13 +778,15 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   // GEMM 3: out = H_hi V + H_lo V
   g.N = d_model;
   g.K = d_ff;
-  g.tiles_n = (d_model + BN - 1) / BN;
+  const bool wide3 = prefill_gemm3_wide(T, d_model, num_sms);
+  g.tiles_n = wide3 ? (d_model + 2 * BN - 1) / (2 * BN) : (d_model + BN - 1) / BN;
   g.nkb = (d_ff + BK - 1) / BK;
   g.split_k = splits;
   g.kb_per_split = (g.nkb + splits - 1) / splits;
   g.units = g.tiles_m * g.tiles_n * splits;
   // GEMM 3 takes h_hi / h_lo by bulk copies of whole blocks: no tensor maps for A
-  e = launch_gemm<kEpiOut, true, true, 4>(tv, tv, tv, tv, g, num_sms, stream);
+  e = wide3 ? launch_gemm<kEpiOut, true, true, 3, true>(tv, tv, tv, tv, g, num_sms, stream)
+            : launch_gemm<kEpiOut, true, true, 4>(tv, tv, tv, tv, g, num_sms, stream);
   if (e != cudaSuccess) return e;
   if (splits > 1) {
     const size_t n4 = static_cast<size_t>(T) * d_model / 4;

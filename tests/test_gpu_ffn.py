@@ -93,6 +93,14 @@ def test_prefill_wide_predictor_ragged_last_unit():
     run_parity(512, 256, 2496, 200, T=T, layer=77, sample_tokens=sample)
 
 
+def test_prefill_wide_output_gemm_ragged_model_width():
+    """Enough token tiles for the 128 x 256 output units; d_model = 1088 leaves the last unit one
+    64-column box of V inside the matrix and one wholly outside it."""
+    T = 1536
+    sample = np.arange(0, T, 61)
+    run_parity(1088, 512, 2048, 160, T=T, layer=78, sample_tokens=sample)
+
+
 @pytest.mark.parametrize("shape", [
     (264, 136, 1001, 80, 3),    # ragged d_ff: last CTA owns one neuron
     (64, 32, 200, 17, 2),       # tiny, few CTAs
