@@ -17,8 +17,9 @@
 //     ahead of it on the stream.  With weight overlap on, P is launched while
 //     the previous call's kernels still run, so the K1 stream -- 80% of the
 //     layer's bytes -- hides behind them.  After the wait: q (stack mode:
-//     q = bf16(RMSNorm(h)), formed by every CTA), x row by row (fp32 FMA), and
-//     the slice's moments (mean, M2); x and the moments go to the workspace.
+//     q = bf16(RMSNorm(h)), formed by every CTA), x row by row (fp32 FMA on bf16
+//     operands), and the slice's moments (mean, M2); x and the moments go to
+//     the workspace.
 //  G  CTA c merges all slices' moments in slice order (every CTA derives the
 //     same bits of theta), compacts the active neurons of slice c, reads their
 //     K2 rows (a = K2.q[r:]) and V rows, and writes its fp32 partial output
@@ -149,6 +150,21 @@ struct PgWs {
 };
 
 // ------------------------------------------------------------------------ P
+// c + a.lo * b.lo + a.hi * b.hi for two bf16 pairs, with the mixed-precision
+// FMA of sm_100 (bf16 operands widened exactly, one fp32 rounding per step):
+// the same bits as two fmaf calls on the widened values, without the widening
+// instructions.
+__device__ __forceinline__ float fma_bf16x2_f32(uint32_t a, uint32_t b, float c) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(c)
+      : "r"(a), "r"(b));
+  return c;
+}
+
 // KCH: 16-byte chunks per lane of a K1 row (r <= 256 * KCH).
 template <int KCH>
 __global__ void __launch_bounds__(kPThreads, 1) decode_score_kernel(const PgParams p) {
@@ -228,24 +244,16 @@ __global__ void __launch_bounds__(kPThreads, 1) decode_score_kernel(const PgPara
       const int ch = lane + 32 * m;
       if (ch < nchunk) {
         const uint4 qv = lds128(qs + ch * 8);
-        const float2 q0 = bf16x2_to_float2(qv.x), q1 = bf16x2_to_float2(qv.y);
-        const float2 q2 = bf16x2_to_float2(qv.z), q3 = bf16x2_to_float2(qv.w);
         uint4 kv[kStageRows];
 #pragma unroll
         for (int j = 0; j < kStageRows; ++j) kv[j] = lds128(kst + static_cast<size_t>(j) * p.r + ch * 8);
 #pragma unroll
         for (int j = 0; j < kStageRows; ++j) {
-          const float2 a = bf16x2_to_float2(kv[j].x), b = bf16x2_to_float2(kv[j].y);
-          const float2 c2 = bf16x2_to_float2(kv[j].z), d = bf16x2_to_float2(kv[j].w);
           float t = acc[j];
-          t = fmaf(a.x, q0.x, t);
-          t = fmaf(a.y, q0.y, t);
-          t = fmaf(b.x, q1.x, t);
-          t = fmaf(b.y, q1.y, t);
-          t = fmaf(c2.x, q2.x, t);
-          t = fmaf(c2.y, q2.y, t);
-          t = fmaf(d.x, q3.x, t);
-          t = fmaf(d.y, q3.y, t);
+          t = fma_bf16x2_f32(kv[j].x, qv.x, t);
+          t = fma_bf16x2_f32(kv[j].y, qv.y, t);
+          t = fma_bf16x2_f32(kv[j].z, qv.z, t);
+          t = fma_bf16x2_f32(kv[j].w, qv.w, t);
           acc[j] = t;
         }
       }
@@ -331,8 +339,9 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
   int* misc_i = reinterpret_cast<int*>(smem + L.misc);
   float* misc_f = reinterpret_cast<float*>(smem + L.misc) + 8;
 
-  // R of this call may now be scheduled; this grid waits for P of this call.
-  griddep_launch_dependents();
+  // This grid waits for P of this call.  R of this call (and through it the next
+  // call's P, whose K1 stream fills the memory queues) is released only once
+  // this CTA's V-row loads are issued, below.
   griddep_wait();
 
   const int n0 = c * p.rpc;
@@ -388,6 +397,7 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
   __syncthreads();
   const int nact = misc_i[0];
   const float theta = misc_f[0];
+  if (nact == 0) griddep_launch_dependents();
   if (c == 0 && tid == 0 && p.theta_out != nullptr) p.theta_out[0] = theta;
   if (p.active_out != nullptr)
     for (int i = tid; i < nr; i += kGThreads) p.active_out[n0 + i] = xs[i] > theta ? 1 : 0;
@@ -411,6 +421,7 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
                        ? ldg_ro128(p.V + static_cast<size_t>(act_i[j0 + u]) * D + ch * 8)
                        : make_uint4(0, 0, 0, 0);
       }
+    if (j0 == 0) griddep_launch_dependents();
     if (j0 == 0) {
       // ... while the warps form h = GELU(x - theta) a, a = <K2[i,:], q[r:]>:
       // two rows per warp, all of both rows' loads issued before the arithmetic
