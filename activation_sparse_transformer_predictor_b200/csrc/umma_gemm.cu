@@ -545,6 +545,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   }
 
   // ------------------------------------------------------------ teardown
+  // Warps 0 and 1 diverged (lane 0 produced / issued, lanes 1-31 came straight
+  // here): reconverge them first, since __syncthreads is an aligned barrier that
+  // every lane of a warp must reach together.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
