@@ -150,21 +150,6 @@ struct PgWs {
 };
 
 // ------------------------------------------------------------------------ P
-// c + a.lo * b.lo + a.hi * b.hi for two bf16 pairs, with the mixed-precision
-// FMA of sm_100 (bf16 operands widened exactly, one fp32 rounding per step):
-// the same bits as two fmaf calls on the widened values, without the widening
-// instructions.
-__device__ __forceinline__ float fma_bf16x2_f32(uint32_t a, uint32_t b, float c) {
-  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
-      "mov.b32 {al, ah}, %1;\n\t"
-      "mov.b32 {bl, bh}, %2;\n\t"
-      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
-      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
-      : "+f"(c)
-      : "r"(a), "r"(b));
-  return c;
-}
-
 // KCH: 16-byte chunks per lane of a K1 row (r <= 256 * KCH).
 template <int KCH>
 __global__ void __launch_bounds__(kPThreads, 1) decode_score_kernel(const PgParams p) {

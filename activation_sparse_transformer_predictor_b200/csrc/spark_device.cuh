@@ -241,20 +241,27 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
   return r;
 }
 
-// acc + <a, b> over 8 bf16 pairs, in a fixed order (fp32 FMA).
+// c + a.lo * b.lo + a.hi * b.hi for two bf16 pairs, with the mixed-precision
+// FMA of sm_100 (bf16 operands widened exactly, one fp32 rounding per step):
+// the same bits as two fmaf calls on the widened values, without the widening
+// instructions.
+__device__ __forceinline__ float fma_bf16x2_f32(uint32_t a, uint32_t b, float c) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(c)
+      : "r"(a), "r"(b));
+  return c;
+}
+
+// acc + <a, b> over 8 bf16 pairs, in a fixed order (fp32 FMA, element 0 first).
 __device__ __forceinline__ float dot8_bf16(uint4 a, uint4 b, float acc) {
-  float2 a0 = bf16x2_to_float2(a.x), b0 = bf16x2_to_float2(b.x);
-  acc = fmaf(a0.x, b0.x, acc);
-  acc = fmaf(a0.y, b0.y, acc);
-  float2 a1 = bf16x2_to_float2(a.y), b1 = bf16x2_to_float2(b.y);
-  acc = fmaf(a1.x, b1.x, acc);
-  acc = fmaf(a1.y, b1.y, acc);
-  float2 a2 = bf16x2_to_float2(a.z), b2 = bf16x2_to_float2(b.z);
-  acc = fmaf(a2.x, b2.x, acc);
-  acc = fmaf(a2.y, b2.y, acc);
-  float2 a3 = bf16x2_to_float2(a.w), b3 = bf16x2_to_float2(b.w);
-  acc = fmaf(a3.x, b3.x, acc);
-  acc = fmaf(a3.y, b3.y, acc);
+  acc = fma_bf16x2_f32(a.x, b.x, acc);
+  acc = fma_bf16x2_f32(a.y, b.y, acc);
+  acc = fma_bf16x2_f32(a.z, b.z, acc);
+  acc = fma_bf16x2_f32(a.w, b.w, acc);
   return acc;
 }
 
