@@ -3,15 +3,15 @@
 // Spark Transformer notes, 关键设计 / "Spark FFN" and "Statistical Top-k", for T
 // tokens at once:
 //   GEMM 1  X = Q1 K1^T                 (predictor; x = K1^T q[:r] per token)
-//           epilogue: per-(token, 128-neuron tile) moments of x (x itself is
-//           stored only for the debug entry point)
-//   theta   per token: merge the tile moments, theta = mean + std Q(1 - k/d_ff)
-//   GEMM 2  X = Q1 K1^T and A = Q2 K2^T  into two TMEM accumulators in one k-loop
-//           (x is recomputed on the tensor cores with the same instruction
-//           sequence as GEMM 1, so its bits are the same, instead of a 36 KB
-//           per token round trip through HBM)
-//           epilogue: h = GELU(max(x - theta, 0)) * a on x > theta, else 0, and
-//           split h = h_hi + h_lo into two bf16 matrices (h_lo = bf16(h - h_hi))
+//           epilogue: x stored once, fp32, in 128 x 128 tiles, and the
+//           per-(token, 128-neuron tile) moments of x
+//   GEMM 2  A = Q2 K2^T
+//           epilogue: theta per token from the tile moments, theta = mean +
+//           std Q(1 - k/d_ff) (merged by the epilogue warps while the main loop
+//           runs up to 64 tokens, else by theta_kernel before); then
+//           h = GELU(max(x - theta, 0)) * a on x > theta, else 0, with x read
+//           back from GEMM 1's tiles, split h = h_hi + h_lo into two bf16
+//           matrices (h_lo = bf16(h - h_hi))
 //   GEMM 3  out = H_hi V + H_lo V        (V read once per k-block for both halves)
 //           epilogue: bf16 out, or fp32 split-K partials reduced in fixed order.
 //
@@ -25,8 +25,8 @@
 // SM), warp 0 = TMA producer (128B-swizzled K-major tiles; V is read N-major),
 // warp 1 = TMEM allocator and single-thread tcgen05.mma issuer (M 128, N 128,
 // K 16 per instruction, fp32 accumulators in TMEM, two accumulators so that
-// the epilogue of one tile overlaps the main loop of the next), warps 2-5 =
-// epilogue (tcgen05.ld, 32 TMEM lanes each).  Every wait is bounded.
+// the epilogue of one tile overlaps the main loop of the next), the remaining
+// warps = epilogue (tcgen05.ld, 32 TMEM lanes per warp).  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -58,7 +58,9 @@ struct GemmParams {
   int xt_tiles_n;         // 128-column tiles per 128-row band of Xt
   float2* moments;        // [M][mom_stride] (mean, M2) of each 128-neuron tile
   int mom_stride;         // 128-neuron tiles per row of moments
-  const float* theta;     // [M]
+  const float* theta;     // [M] thresholds from theta_kernel, or nullptr: GEMM 2's epilogue derives them
+  float Q;                // standard-normal quantile Q(1 - k/d_ff) of the threshold
+  float* theta_out;       // optional [M]: the thresholds GEMM 2 derived (debug entry point)
   uint16_t* h_hi;         // bf16, blocked: see h_block()
   uint16_t* h_lo;         // bf16, blocked like h_hi
   int h_kb;               // 64-neuron blocks per 128-token band of h_hi / h_lo
@@ -200,6 +202,54 @@ __device__ __forceinline__ float4 gate_x(const GemmParams& p, const float4* tile
   return nb + 4 * i < p.N ? __ldcg(tile + i * BM + row) : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// theta of token m from the per-(token, 128-neuron tile) moments of GEMM 1: the
+// four gate epilogue warps that share TMEM lane quarter `quarter` (and so this
+// row) each merge a quarter of the tiles, weighted mean first, then
+// M2 = sum_j M2_j + n_j (mean_j - mean)^2; the partials are combined through
+// shared memory (tred, 8 x 128 floats) in warp order, so every warp gets the
+// same bits.  All four warps must call it.
+__device__ __forceinline__ float gate_theta(const GemmParams& p, int m, int row, int colgrp, int quarter,
+                                            float* tred) {
+  const int tiles = p.mom_stride;
+  const int j0 = colgrp * tiles / 4, j1 = (colgrp + 1) * tiles / 4;
+  const bool ok = m < p.M;
+  const float2* mr = p.moments + static_cast<size_t>(ok ? m : 0) * p.mom_stride;
+  // loads in batches of 8, all of a batch in flight before its arithmetic
+  constexpr int kB = 8;
+  float s = 0.f;
+  for (int jb = j0; jb < j1; jb += kB) {
+    float2 mm[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) mm[u] = (ok && jb + u < j1) ? mr[jb + u] : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kB; ++u)
+      if (jb + u < j1) s = fmaf(static_cast<float>(min(BN, p.N - (jb + u) * BN)), mm[u].x, s);
+  }
+  tred[colgrp * BM + row] = s;
+  named_bar_sync(1 + quarter, 128);
+  const float mean = (((tred[row] + tred[BM + row]) + tred[2 * BM + row]) + tred[3 * BM + row]) / static_cast<float>(p.N);
+  float m2 = 0.f;
+  for (int jb = j0; jb < j1; jb += kB) {
+    float2 mm[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u) mm[u] = (ok && jb + u < j1) ? mr[jb + u] : make_float2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kB; ++u)
+      if (jb + u < j1) {
+        const float d = mm[u].x - mean;
+        m2 += mm[u].y + static_cast<float>(min(BN, p.N - (jb + u) * BN)) * d * d;
+      }
+  }
+  tred[(4 + colgrp) * BM + row] = m2;
+  named_bar_sync(1 + quarter, 128);
+  const float M2 = ((tred[4 * BM + row] + tred[5 * BM + row]) + tred[6 * BM + row]) + tred[7 * BM + row];
+  return fmaf(sqrtf(fmaxf(M2, 0.f) / static_cast<float>(p.N)), p.Q, mean);
+}
+
 // WIDE (GEMMs 1 and 2): a unit is 128 rows x 256 columns: each stage holds one
 // A tile and two adjacent 128-row B tiles, and each K 16 step is one M 128 x
 // N 256 instruction into 256 TMEM columns.
@@ -222,6 +272,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   uint64_t* tempty = tfull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* tred = reinterpret_cast<float*>(smem + STAGES * kStageBytes + 256);  // GEMM 2: theta partials
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   DeviceControl* ctl = p.ctl;
@@ -388,10 +439,18 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       const int gtile_nb = n_base + gcol / BN * BN;       // first column of its score tile
       const int gx0 = gcol % BN / 4;                      // its first float4 group in that tile
       float4 xr[EPI == kEpiGate ? kGateCols / 4 : 1];
+      float th = 0.f;
       if (EPI == kEpiGate) {
         const float4* t0 = xt_tile(p, tm, gtile_nb);
 #pragma unroll
         for (int i = 0; i < kGateCols / 4; ++i) xr[i] = gate_x(p, t0, row, gtile_nb, gx0 + i);
+        if (WIDE || p.theta != nullptr) {  // wide units: always several per CTA, theta_kernel ran
+          th = row_ok ? p.theta[m] : 0.f;
+        } else {
+          // the threshold of this row, while the accumulator is still being formed
+          th = gate_theta(p, m, row, colgrp, quarter, tred);
+          if (p.theta_out != nullptr && colgrp == 0 && row_ok) p.theta_out[m] = th;
+        }
       }
       if (!mbar_wait_bounded(&tfull[acc], uses[acc] & 1u, p.wait_limit_ns, ctl, 120) || *abort_flag) {
         *abort_flag = 1;
@@ -454,7 +513,6 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           if (row_ok && nb < p.N) p.moments[static_cast<size_t>(m) * p.mom_stride + nb / BN] = make_float2(mean, m2);
         }
       } else if (EPI == kEpiGate) {
-        const float th = row_ok ? p.theta[m] : 0.f;
         {
           const int nb = n_base + gcol;
           const uint32_t ta = taddr + static_cast<uint32_t>(gcol);
@@ -646,7 +704,7 @@ template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const CUtensorMap& b2,
                         const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes * (WIDE ? 2 : 1);
-  constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256;
+  constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256 + (EPI == kEpiGate ? 8 * BM * 4 : 0);
   auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE>;
   static int set_dev = -1;
   int dev = 0;
@@ -732,7 +790,9 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   g.xt_tiles_n = tiles_n;
   g.moments = moments;
   g.mom_stride = tiles_n;
-  g.theta = theta;
+  g.theta = nullptr;
+  g.Q = a.Q;
+  g.theta_out = a.theta_out;
   g.h_hi = h_hi;
   g.h_lo = h_lo;
   g.h_kb = h_kb;
@@ -762,10 +822,20 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
     e = launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
   }
   if (e != cudaSuccess) return e;
-  theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, tiles_n, a.Q, theta, a.theta_out);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // GEMM 2: A = Q2 K2^T; the gate h = GELU(max(x - theta, 0)) a with x as GEMM 1
   // stored it, split into h_hi + h_lo.  Wide units under the same rule as GEMM 1.
+  // Up to 64 tokens the epilogue warps derive theta from the tile moments while
+  // the main loop runs, which saves theta_kernel and one kernel boundary
+  // (measured 47.4 -> 45.0 us per call at T = 16, 45.4 -> 44.6 at T = 64).  Every
+  // CTA of a token band repeats that merge for the same rows, which at T = 256
+  // (72 CTAs per band, 256 rows) cost more than it saved (+6 us), and with several
+  // units per CTA it would sit between units: there theta_kernel runs first.
+  const int gate_units = wide_units >= num_sms ? wide_units : g.tiles_m * tiles_n;
+  if (T > 64 || wide_units >= num_sms || gate_units > num_sms) {
+    theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, tiles_n, a.Q, theta, a.theta_out);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    g.theta = theta;
+  }
   g.K = d2;
   g.nkb = (d2 + BK - 1) / BK;
   g.kb_per_split = g.nkb;
