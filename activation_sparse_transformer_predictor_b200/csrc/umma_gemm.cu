@@ -253,15 +253,23 @@ __device__ __forceinline__ float gate_theta(const GemmParams& p, int m, int row,
 // WIDE (GEMMs 1 and 2): a unit is 128 rows x 256 columns: each stage holds one
 // A tile and two adjacent 128-row B tiles, and each K 16 step is one M 128 x
 // N 256 instruction into 256 TMEM columns.
-template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false>
+// A64 (GEMMs 1 and 2, at most 64 tokens): each stage holds only the 64 token
+// rows that exist (an 8 KB A box) and the B tile right after it; the M 128
+// instruction still reads 128 A rows, its rows 64..127 coming from the B tile's
+// bytes, which only ever reach accumulator rows >= 64 -- rows no token owns,
+// which the epilogue skips.  The 24 KB stages let 8 of them (128 KB of weights)
+// be in flight instead of 6 (96 KB).
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false, bool A64 = false>
 __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
                      const GemmParams p) {
   static_assert(!WIDE || B_NMAJOR == (EPI == kEpiOut), "wide GEMM 3 takes V N-major; GEMMs 1 and 2 K-major");
   static_assert(!DUAL || EPI == kEpiOut, "two A operands (h_hi, h_lo) are GEMM 3's");
+  static_assert(!A64 || (EPI != kEpiOut && !WIDE), "64-row A boxes: narrow GEMMs 1 and 2 only");
   constexpr int kBTiles = WIDE ? 2 : 1;
-  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes * kBTiles;
+  constexpr int kAB = A64 ? kABytes / 2 : kABytes;  // bytes of one stage's A box
+  constexpr int kStageBytes = kAB * (DUAL ? 2 : 1) + kBBytes * kBTiles;
   constexpr int kAccCols = WIDE ? 2 * BN : BN;  // TMEM columns of one tile's accumulators
   constexpr int kTmemCols = 2 * kAccCols;       // double buffered
   extern __shared__ unsigned char smem_raw[];
@@ -320,7 +328,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         }
         unsigned char* sa = smem + stage * kStageBytes;
         mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        unsigned char* sb = sa + kABytes * (DUAL ? 2 : 1);
+        unsigned char* sb = sa + kAB * (DUAL ? 2 : 1);
         if (EPI == kEpiOut) {
           // h_hi and h_lo blocks: already in the operand layout
           bulk_g2s(sa, h_block(p.h_hi, p, tm, kb), kHBlockBytes, &full[stage]);
@@ -396,7 +404,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         }
         tc_fence_after();
         const uint32_t sa = smem_u32(smem + stage * kStageBytes);
-        const uint32_t sb = sa + kABytes * (DUAL ? 2 : 1);
+        const uint32_t sb = sa + kAB * (DUAL ? 2 : 1);
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k) {
           const uint64_t bdesc = B_NMAJOR ? desc_nmajor_sw128(sb + k * 16 * 128, kBBytes / 2)
@@ -700,12 +708,12 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false>
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false, bool A64 = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const CUtensorMap& b2,
                         const GemmParams& p, int num_sms, cudaStream_t stream) {
-  constexpr int kStageBytes = kABytes * (DUAL ? 2 : 1) + kBBytes * (WIDE ? 2 : 1);
+  constexpr int kStageBytes = (A64 ? kABytes / 2 : kABytes) * (DUAL ? 2 : 1) + kBBytes * (WIDE ? 2 : 1);
   constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256 + (EPI == kEpiGate ? 8 * BM * 4 : 0);
-  auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE>;
+  auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE, A64>;
   static int set_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -776,7 +784,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   const uint16_t* q = static_cast<const uint16_t*>(a.q);
   CUtensorMap tq1, tq2, tk1, tk2, tv;
   const uint64_t qrow = static_cast<uint64_t>(d_model) * 2;
-  if (!make_tmap(&tq1, q, r, T, qrow, BK, BM) || !make_tmap(&tq2, q + r, d2, T, qrow, BK, BM) ||
+  // up to 64 tokens the token operand is fetched as 64-row boxes (A64 above)
+  const bool a64 = T <= 64;
+  const uint32_t qbox = a64 ? 64 : BM;
+  if (!make_tmap(&tq1, q, r, T, qrow, BK, qbox) || !make_tmap(&tq2, q + r, d2, T, qrow, BK, qbox) ||
       !make_tmap(&tk1, a.K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, BN) ||
       !make_tmap(&tk2, a.K2, d2, d_ff, static_cast<uint64_t>(d2) * 2, BK, BN) ||
       !make_tmap(&tv, a.V, d_model, d_ff, static_cast<uint64_t>(d_model) * 2, 64, BK))
@@ -818,6 +829,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
     g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
     g.units = wide_units;
     e = launch_gemm<kEpiPredictor, false, false, 4, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  } else if (a64) {
+    e = launch_gemm<kEpiPredictor, false, false, 8, false, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
   } else {
     e = launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
   }
@@ -846,7 +859,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   } else {
     g.tiles_n = tiles_n;
     g.units = g.tiles_m * g.tiles_n;
-    e = launch_gemm<kEpiGate, false, false, 6>(tq2, tq2, tk2, tk2, g, num_sms, stream);
+    e = a64 ? launch_gemm<kEpiGate, false, false, 8, false, true>(tq2, tq2, tk2, tk2, g, num_sms, stream)
+            : launch_gemm<kEpiGate, false, false, 6>(tq2, tq2, tk2, tk2, g, num_sms, stream);
   }
   if (e != cudaSuccess) return e;
   // GEMM 3: out = H_hi V + H_lo V
