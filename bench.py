@@ -37,6 +37,8 @@ sys.path.insert(0, ROOT)
 D_MODEL, R, D_FF, K = 2304, 1152, 9216, 737
 N_COPIES = 16
 METRIC = "Spark-FFN tokens/s per layer (T=1, 256) and achieved HBM GB/s vs ~8 TB/s"
+DECODE_WORKLOAD = "Gemma-2-2B-shaped Spark FFN layer, decode T=1 (one token per step)"
+WEIGHTS_RECIPE = "bf16 ~N(0,1/fan_in), q ~N(0,1), seed 1234"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
@@ -273,8 +275,8 @@ def run_reference(args):
     line = {"metric": METRIC, "value": v, "unit": "tokens/s", "impl": "reference", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "Gemma-2-2B-shaped Spark FFN layer, decode T=1", "d_model": D_MODEL, "r": R,
-                       "d_ff": D_FF, "k": K, "tokens_per_step": 1},
+            "config": {"workload": DECODE_WORKLOAD, "d_model": D_MODEL, "r": R, "d_ff": D_FF, "k": K,
+                       "tokens_per_step": 1, "weights": WEIGHTS_RECIPE, "parallelism": f"replicas x{args.gpus}"},
             "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": f"{args.steps} decode tokens, one per step, single thread"},
             "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -432,9 +434,9 @@ def main():
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": n_timed,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "Gemma-2-2B-shaped Spark FFN layer, decode T=1 (one token per step)",
+            "config": {"workload": DECODE_WORKLOAD,
                        "d_model": D_MODEL, "r": R, "d_ff": D_FF, "k": K, "tokens_per_step": 1,
-                       "active_neurons": m_active, "weights": "bf16 ~N(0,1/fan_in), q ~N(0,1), seed 1234",
+                       "active_neurons": m_active, "weights": WEIGHTS_RECIPE,
                        "l2": f"inputs larger than L2: steps cycle over {N_COPIES} weight copies "
                              f"({N_COPIES * 2 * D_MODEL * D_FF * 2 / 1e9:.2f} GB)",
                        "timing": "CUDA graph of 128 library calls replayed; CUDA events on the launch stream",
