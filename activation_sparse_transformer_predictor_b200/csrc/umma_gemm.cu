@@ -22,11 +22,13 @@
 // rounding and break the 2e-3 relative-L2 target.
 //
 // One kernel template serves the three GEMMs: a persistent grid (one CTA per
-// SM), warp 0 = TMA producer (128B-swizzled K-major tiles; V is read N-major),
-// warp 1 = TMEM allocator and single-thread tcgen05.mma issuer (M 128, N 128,
-// K 16 per instruction, fp32 accumulators in TMEM, two accumulators so that
-// the epilogue of one tile overlaps the main loop of the next), the remaining
-// warps = epilogue (tcgen05.ld, 32 TMEM lanes per warp).  Every wait is bounded.
+// SM), warp 0 = producer (TMA copies of 128B-swizzled K-major tiles, V read
+// N-major; GEMM 3's h blocks by 1-D bulk copies, already in operand order),
+// warp 1 = TMEM allocator and single-thread tcgen05.mma issuer (M 128, N 128 or
+// 256, K 16 per instruction, fp32 accumulators in TMEM, two accumulators so
+// that the epilogue of one tile overlaps the main loop of the next), the
+// remaining warps = epilogue (tcgen05.ld, 32 TMEM lanes per warp).  Every wait
+// is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
