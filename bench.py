@@ -453,7 +453,7 @@ def main():
             "e2e": {"value": whole_job_rate(1, e2e_ms, world), "unit": "tokens/s", "h2d_bytes_per_step": D_MODEL * 2,
                     "d2h_bytes_per_step": D_MODEL * 2,
                     "path": "public Python API per step: pinned q H2D copy, ffn_forward, out D2H copy"},
-            "gpu_launches": 2 * n_timed,
+            "gpu_launches": 3 * n_timed,  # score, gather and reduce kernel per timed call
             "clocks": clk.summary(),
             "also": also,
         }
