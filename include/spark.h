@@ -112,9 +112,10 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
  *           both 16-byte aligned
  *   K1s, K2s, Vs : HOST arrays of n_layers DEVICE pointers, each as in spark_ffn_forward
  *   q_dbg, out_dbg : optional bf16 [n_layers][d_model]: every q_l and SparkFFN_l(q_l)
- * One launch of the single-token kernel per layer; each launch forms q_l from h_l
- * itself and writes h_{l+1}.  Requires the single-token kernel to support the
- * shape (the Gemma-2-2B shape does), else SPARK_EINVAL.
+ * Each layer runs the single-token kernel chain (score, gather, reduce): the
+ * score kernel forms q_l from h_l itself and the reduce kernel writes h_{l+1}.
+ * Requires the single-token kernels to support the shape (the Gemma-2-2B shape
+ * does), else SPARK_EINVAL.
  */
 SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void* const* K1s,
                                      const void* const* K2s, const void* const* Vs, int n_layers,
@@ -191,8 +192,9 @@ SPARK_API int spark_set_wait_limit_ns(unsigned long long ns);
 
 /*
  * Single-token decode (spark_ffn_forward, and _tokens / _debug with one token)
- * runs as two kernels: a score kernel (x, its moments) and a gather kernel
- * (theta, the active K2 / V rows, out).  With weight overlap enabled (nonzero),
+ * runs as three kernels: a score kernel (x, its moments), a gather kernel
+ * (theta, the active K2 / V rows, partial outputs) and a reduce kernel (out).
+ * With weight overlap enabled (nonzero),
  * the score kernel is launched as a programmatic dependent of whatever kernel
  * precedes the call on the stream: it starts streaming K1 into shared memory
  * while that kernel is still running, and reads q, and writes anything, only
