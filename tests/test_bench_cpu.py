@@ -29,3 +29,26 @@ def test_reference_arm_json_line(capsys, monkeypatch):
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_profile_traffic_tracks_the_kernel_sources(tmp_path, monkeypatch):
+    """The roofline's DRAM traffic comes from a committed ncu summary only while the
+    kernel sources still hash to the value recorded with it; otherwise it is null."""
+    # the committed summaries match the committed sources
+    assert bench.profile_traffic("ffn_decode_pg_gemma_T1.txt", bench.DECODE_SOURCES) > 0
+    assert bench.profile_traffic("stat_topk_32768x4096.txt", bench.TOPK_SOURCES) > 0
+    # a copy of the tree in which one source changed: the summary no longer applies
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    for rel in bench.DECODE_SOURCES:
+        dst = root / rel
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        dst.write_bytes(open(os.path.join(ROOT, rel), "rb").read())
+    summary = open(os.path.join(ROOT, "profiles", "ffn_decode_pg_gemma_T1.txt")).read()
+    (root / "profiles" / "ffn_decode_pg_gemma_T1.txt").write_text(summary)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.profile_traffic("ffn_decode_pg_gemma_T1.txt", bench.DECODE_SOURCES) > 0
+    src = root / bench.DECODE_SOURCES[0]
+    src.write_bytes(src.read_bytes() + b"\n// changed\n")
+    assert bench.profile_traffic("ffn_decode_pg_gemma_T1.txt", bench.DECODE_SOURCES) is None
+    assert bench.profile_traffic("no_such_summary.txt", bench.DECODE_SOURCES) is None
