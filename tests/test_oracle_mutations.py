@@ -20,6 +20,8 @@ MUTATIONS = {
     "theta_sign": ("return mean + sd * oracle_topk_quantile", "return mean - sd * oracle_topk_quantile"),
     "variance_drops_mean": ("double c = x[i] - mean;", "double c = x[i];"),
     "gelu_cubic_term": ("0.044715 * s * s * s", "0.044715 * s * s"),
+    "gelu_truncated_constant": ("sqrt(2.0 / M_PI)", "0.7979"),
+    "gelu_cubic_coefficient": ("0.044715 * s * s * s", "0.04472 * s * s * s"),
     "bisection_direction": ("lo = mid; /* too much", "hi = mid; /* too much"),
     "a_uses_q_head": ("* oracle_bf16_to_f64(qt[r + j])", "* oracle_bf16_to_f64(qt[j])"),
     "K1_transposed": ("K1[i * r + j]", "K1[j * r + i]"),

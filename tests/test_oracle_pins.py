@@ -165,6 +165,41 @@ def test_gelu_forms():
     assert oracle.gelu(30.0) == pytest.approx(30.0, rel=1e-15)
 
 
+def _gelu_tanh_decimal(s: str, digits: int = 50):
+    """GELU, tanh form, evaluated as s / (1 + exp(-2u)), u = sqrt(2/pi) (s + 0.044715 s^3), in
+    `digits`-digit decimal arithmetic with pi from Machin's formula 16 atan(1/5) - 4 atan(1/239).
+    A different route from the oracle's (no tanh, no libm constant), exact to far below fp64."""
+    from decimal import Decimal, localcontext
+
+    def atan_inv(n):
+        x = Decimal(1) / n
+        term, total, k = x, x, 1
+        while True:
+            term *= -x * x
+            k += 2
+            if abs(term / k) < Decimal(10) ** -(digits - 2):
+                return total
+            total += term / k
+
+    with localcontext() as ctx:
+        ctx.prec = digits
+        pi = 16 * atan_inv(5) - 4 * atan_inv(239)
+        v = Decimal(s)
+        u = (Decimal(2) / pi).sqrt() * (v + Decimal("0.044715") * v ** 3)
+        return float(v / (1 + (-2 * u).exp()))
+
+
+def test_gelu_tanh_closed_form_values():
+    # closed-form values: GELU_tanh(1) = 0.8411919906, GELU_tanh(2) = 1.9545976941 (to 10 digits)
+    assert oracle.gelu(1.0) == pytest.approx(0.8411919906, abs=1e-10)
+    assert oracle.gelu(2.0) == pytest.approx(1.9545976941, abs=1e-10)
+    # the same points and more, to full double precision, from the 50-digit evaluation
+    assert oracle.gelu(1.0) == pytest.approx(0.8411919906082768, rel=1e-14)
+    assert oracle.gelu(2.0) == pytest.approx(1.954597694087775, rel=1e-14)
+    for s in ("0.5", "1", "2", "3", "-1.5", "0.125", "4.75"):
+        assert oracle.gelu(float(s)) == pytest.approx(_gelu_tanh_decimal(s), rel=1e-13, abs=1e-300), s
+
+
 # ---------------------------------------------------------------- FFN
 def _layer(rng, d_model, r, d_ff, T):
     K1 = _to_bf16_bits(rng.standard_normal((d_ff, r)) / math.sqrt(r))
