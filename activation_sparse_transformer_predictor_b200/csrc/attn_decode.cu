@@ -339,9 +339,6 @@ cudaError_t launch_attn_decode(const AttnArgs& a, int num_sms, cudaStream_t stre
     cudaGetLastError();
   }
   int cs = (cs16_ok[dev] == 1 && a.n_ctx >= 16 * 32) ? 16 : 8;
-  // SPARK_ATTN_CLUSTER=8 (test / tuning knob) forces the portable cluster size
-  const char* env = std::getenv("SPARK_ATTN_CLUSTER");
-  if (env != nullptr && std::atoi(env) == 8) cs = 8;
   AttnParams p;
   p.q = static_cast<const uint16_t*>(a.q);
   p.K = static_cast<const uint16_t*>(a.K);

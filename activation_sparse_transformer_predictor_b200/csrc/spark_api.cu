@@ -19,25 +19,13 @@ namespace {
 constexpr unsigned long long kDefaultWaitLimitNs = 1000000000ull;  // one second
 unsigned long long g_wait_limit_ns = kDefaultWaitLimitNs;
 
-// Speculative L2 prefetch margin of the decode kernel, in units of the local
-// standard deviation below the threshold (0 disables).  SPARK_SPEC_MARGIN
-// overrides it (tuning knob).
-float spec_margin_default() {
-  const char* e = std::getenv("SPARK_SPEC_MARGIN");
-  return e ? static_cast<float>(std::atof(e)) : 0.35f;
-}
-float g_spec_margin = spec_margin_default();
+// Speculative L2 prefetch margin of the fused small-batch kernel, in units of
+// the local standard deviation below the threshold.
+constexpr float kSpecMargin = 0.35f;
 
 // Single-token decode: whether the score kernel may stream K1 before the work
 // ahead of it on the stream has completed (spark_set_weight_overlap).
 bool g_weight_overlap = false;
-
-// Tuning / test knob read per call: SPARK_DECODE_IMPL=exchange selects the
-// one-launch exchange kernel instead of the score + gather pair.
-bool decode_use_exchange_kernel() {
-  const char* e = std::getenv("SPARK_DECODE_IMPL");
-  return e != nullptr && std::strcmp(e, "exchange") == 0;
-}
 
 
 struct DeviceInfo {
@@ -189,7 +177,7 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
     return SPARK_OK;
   }
 
-  if (T == 1 && never_arrive == 0 && !decode_use_exchange_kernel()) {
+  if (T == 1 && never_arrive == 0) {
     const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin);
     if (pp.ok) {
       void* ws = nullptr;
@@ -212,41 +200,6 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
       a.wait_limit_ns = g_wait_limit_ns;
       a.overlap_weights = g_weight_overlap;
       if (launch_decode_pg(pp, a, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return SPARK_ECUDA;
-      }
-      return SPARK_OK;
-    }
-  }
-
-  if (T == 1) {
-    // SPARK_DECODE_CAP (test / tuning knob): speculative candidates per CTA.
-    const char* capenv = std::getenv("SPARK_DECODE_CAP");
-    const int cap_override = capenv ? std::atoi(capenv) : -1;
-    const DecodePlan dp = plan_decode(d_model, r, d_ff, di.num_sms, di.smem_optin, cap_override);
-    if (dp.ok) {
-      void* ws = nullptr;
-      const int wst = get_workspace(dev, stream, dp.ws_bytes, &ws);
-      if (wst != SPARK_OK) return wst;
-      FusedArgs a;
-      a.q = q;
-      a.K1 = K1;
-      a.K2 = K2;
-      a.V = V;
-      a.out = out;
-      a.T = 1;
-      a.d_model = d_model;
-      a.r = r;
-      a.d_ff = d_ff;
-      a.Q = Q;
-      a.spec_margin = 0.f;
-      a.x_out = x_out;
-      a.theta_out = theta_out;
-      a.active_out = active_out;
-      a.workspace = ws;
-      a.wait_limit_ns = g_wait_limit_ns;
-      a.never_arrive = never_arrive;
-      if (launch_decode(dp, a, stream) != cudaSuccess) {
         cudaGetLastError();
         return SPARK_ECUDA;
       }
@@ -283,7 +236,7 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
     a.r = r;
     a.d_ff = d_ff;
     a.Q = Q;
-    a.spec_margin = g_spec_margin;
+    a.spec_margin = kSpecMargin;
     a.x_out = x_out ? x_out + static_cast<size_t>(t0) * d_ff : nullptr;
     a.theta_out = theta_out ? theta_out + t0 : nullptr;
     a.active_out = active_out ? active_out + static_cast<size_t>(t0) * d_ff : nullptr;
@@ -299,6 +252,9 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
 }
 
 }  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns; }
+
 }  // namespace spark
 
 using namespace spark;
@@ -355,73 +311,34 @@ SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void
   const int dst = device_info(dev, &di);
   if (dst != SPARK_OK) return dst;
   const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d_ff)));
-  if (!decode_use_exchange_kernel()) {
-    const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin);
-    if (!pp.ok) return SPARK_EINVAL;  // shape not supported by the single-token kernels
-    void* ws = nullptr;
-    const int wst = get_workspace(dev, stream, pp.ws_bytes, &ws);
-    if (wst != SPARK_OK) return wst;
-    // every layer's score kernel forms q_l = bf16(RMSNorm(h_l)); its reduce
-    // kernel writes h_{l+1} = h_l + bf16(out_l)
-    for (int l = 0; l < n_layers; ++l) {
-      DecodePgArgs a;
-      a.K1 = K1s[l];
-      a.K2 = K2s[l];
-      a.V = Vs[l];
-      a.out = out_dbg ? static_cast<unsigned char*>(out_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
-      a.d_model = d_model;
-      a.r = r;
-      a.d_ff = d_ff;
-      a.Q = Q;
-      a.q_dbg = q_dbg ? static_cast<unsigned char*>(q_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
-      a.workspace = ws;
-      a.wait_limit_ns = g_wait_limit_ns;
-      // after the first layer, the kernel ahead of each score kernel is this
-      // library's own reduce kernel, which writes no weights
-      a.overlap_weights = l > 0 || g_weight_overlap;
-      a.h_in = l == 0 ? h_in : h_out;
-      a.h_base = a.h_in;
-      a.h_out = h_out;
-      a.eps = eps;
-      if (launch_decode_pg(pp, a, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return SPARK_ECUDA;
-      }
-    }
-    return SPARK_OK;
-  }
-  const char* capenv = std::getenv("SPARK_DECODE_CAP");
-  const DecodePlan dp = plan_decode(d_model, r, d_ff, di.num_sms, di.smem_optin, capenv ? std::atoi(capenv) : -1);
-  if (!dp.ok) return SPARK_EINVAL;  // shape not supported by the single-token kernel
+  const DecodePgPlan pp = plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin);
+  if (!pp.ok) return SPARK_EINVAL;  // shape not supported by the single-token kernels
   void* ws = nullptr;
-  const int wst = get_workspace(dev, stream, dp.ws_bytes, &ws);
+  const int wst = get_workspace(dev, stream, pp.ws_bytes, &ws);
   if (wst != SPARK_OK) return wst;
+  // every layer's score kernel forms q_l = bf16(RMSNorm(h_l)); its reduce
+  // kernel writes h_{l+1} = h_l + bf16(out_l)
   for (int l = 0; l < n_layers; ++l) {
-    FusedArgs a;
-    a.q = nullptr;
+    DecodePgArgs a;
     a.K1 = K1s[l];
     a.K2 = K2s[l];
     a.V = Vs[l];
     a.out = out_dbg ? static_cast<unsigned char*>(out_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
-    a.T = 1;
     a.d_model = d_model;
     a.r = r;
     a.d_ff = d_ff;
     a.Q = Q;
-    a.spec_margin = 0.f;
-    a.x_out = nullptr;
-    a.theta_out = nullptr;
-    a.active_out = nullptr;
+    a.q_dbg = q_dbg ? static_cast<unsigned char*>(q_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
     a.workspace = ws;
     a.wait_limit_ns = g_wait_limit_ns;
-    a.never_arrive = 0;
-    // every CTA reads h before it arrives at the exchange and the column owners
-    // write it after the exchange, so the update is in place from layer 1 on
+    // after the first layer, the kernel ahead of each score kernel is this
+    // library's own reduce kernel, which writes no weights
+    a.overlap_weights = l > 0 || g_weight_overlap;
     a.h_in = l == 0 ? h_in : h_out;
+    a.h_base = a.h_in;
     a.h_out = h_out;
     a.eps = eps;
-    a.q_dbg = q_dbg ? static_cast<unsigned char*>(q_dbg) + static_cast<size_t>(l) * d_model * 2 : nullptr;
-    if (launch_decode(dp, a, stream) != cudaSuccess) {
+    if (launch_decode_pg(pp, a, stream) != cudaSuccess) {
       cudaGetLastError();
       return SPARK_ECUDA;
     }
@@ -506,16 +423,18 @@ SPARK_API int spark_query_status(spark_stream_t stream_) {
   }
   int dev;
   if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  // errors recorded by spark_ffn_forward_noalloc live in its own scratch
+  const int na = noalloc_take_status(dev);
   void* ptr = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     auto it = g_workspaces.find({dev, stream});
-    if (it == g_workspaces.end() || it->second.ptr == nullptr) return SPARK_OK;
+    if (it == g_workspaces.end() || it->second.ptr == nullptr) return na;
     ptr = it->second.ptr;
   }
   DeviceControl ctl;
   if (cudaMemcpy(&ctl, ptr, sizeof ctl, cudaMemcpyDeviceToHost) != cudaSuccess) return SPARK_ECUDA;
-  if (ctl.status == kDevOk && ctl.abort == 0) return SPARK_OK;
+  if (ctl.status == kDevOk && ctl.abort == 0) return na;
   if (cudaMemset(ptr, 0, sizeof ctl) != cudaSuccess) return SPARK_ECUDA;  // barrier state too
   return ctl.status == kDevTimeout ? SPARK_ETIMEOUT : SPARK_ECUDA;
 }

@@ -24,13 +24,10 @@ struct DeviceControl {
   unsigned int exit_count;  // CTAs that finished the current launch
   unsigned int arrive1;     // arrivals at the statistics exchange
   unsigned int arrive2;     // arrivals at the partial-output exchange
-  unsigned int pg_arrive;   // single-token gather kernel: clusters that wrote their partial
-  unsigned int epoch;       // single-token decode launch number on this workspace
+  unsigned int pad0[2];
   unsigned long long theta_word;  // published threshold of token 0 (high word) | flag (low word)
   float theta[8];                 // published thresholds of tokens 1..7
-  unsigned int dec_arrive[2];     // single-token decode: exchange arrivals, by epoch parity
-  unsigned int dec_s0[2];         // single-token decode: first-stage arrivals, by epoch parity
-  unsigned int pad1[10];
+  unsigned int pad1[14];
 };
 static_assert(sizeof(DeviceControl) == 128, "DeviceControl layout");
 

@@ -9,6 +9,16 @@ namespace spark {
 
 struct DeviceControl;
 
+// ---------------------------------------------------------------- library settings
+// Time limit of every device-side wait (spark_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+
+// The no-allocation entry point's fixed scratch on device `dev` (current):
+// if a device error is recorded in its control block, clear the block and
+// return that error (SPARK_ETIMEOUT); SPARK_OK if none, or if the entry point
+// was never set up on `dev`.
+int noalloc_take_status(int dev);
+
 // ---------------------------------------------------------------- stat top-k
 cudaError_t launch_stat_topk(const float* x, float* out, int rows, int d, float Q, cudaStream_t stream);
 
@@ -53,18 +63,6 @@ struct FusedArgs {
 };
 
 cudaError_t launch_fused(const FusedPlan& plan, const FusedArgs& args, cudaStream_t stream);
-
-// ---------------------------------------------------------------- single-token decode (one exchange)
-struct DecodePlan {
-  int grid, rows_per_cta, cap, col_width, n_col_ctas;
-  size_t smem_bytes, ws_bytes;
-  bool ok;
-};
-
-// cap_override >= 0 forces the number of speculative candidates per CTA (0 makes
-// every CTA take the recompute path; used to test it).
-DecodePlan plan_decode(int d_model, int r, int d_ff, int num_sms, size_t smem_optin, int cap_override);
-cudaError_t launch_decode(const DecodePlan& plan, const FusedArgs& args, cudaStream_t stream);
 
 // ---------------------------------------------------------------- single-token decode: score + gather kernels
 struct DecodePgPlan {

@@ -10,6 +10,7 @@
 // device memory up front and treats any later allocation as a failure, or code
 // running where a device allocation could block on or interfere with another
 // allocator.
+#include <cstddef>
 #include <cstdint>
 #include <mutex>
 
@@ -46,6 +47,12 @@ int scratch_address(int dev, void** out) {
   return SPARK_OK;
 }
 
+// Device address of the scratch on `dev` if it was already looked up, else nullptr.
+void* scratch_address_if_set(int dev) {
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  return (dev >= 0 && dev < kMaxDevices) ? g_scratch_addr[dev] : nullptr;
+}
+
 bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 bool ranges_overlap(const void* a, size_t abytes, const void* b, size_t bbytes) {
@@ -54,6 +61,23 @@ bool ranges_overlap(const void* a, size_t abytes, const void* b, size_t bbytes) 
 }
 
 }  // namespace
+
+int noalloc_take_status(int dev) {
+  void* scratch = scratch_address_if_set(dev);
+  if (scratch == nullptr) return SPARK_OK;
+  DeviceControl ctl;
+  if (cudaMemcpy(&ctl, scratch, sizeof ctl, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  if (ctl.status == kDevOk && ctl.abort == 0) return SPARK_OK;
+  if (cudaMemset(scratch, 0, sizeof ctl) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return ctl.status == kDevTimeout ? SPARK_ETIMEOUT : SPARK_ECUDA;
+}
+
 }  // namespace spark
 
 extern "C" SPARK_API int spark_ffn_forward_noalloc(const void* q, const void* K1, const void* K2, const void* V,
@@ -88,9 +112,15 @@ extern "C" SPARK_API int spark_ffn_forward_noalloc(const void* q, const void* K1
   void* scratch = nullptr;
   const int st = scratch_address(dev, &scratch);
   if (st != SPARK_OK) return st;
-  // The counters and flags of the control block must start at zero; the rest
-  // of the scratch is fully written before it is read.
-  if (cudaMemsetAsync(scratch, 0, sizeof(DeviceControl), stream) != cudaSuccess) {
+  // The arrival counters and the published threshold must start at zero (the
+  // last CTA of a completed launch resets them, but a launch that gave up
+  // waiting leaves them set); the rest of the scratch is fully written before
+  // it is read.  The first three words -- the recorded error, the abort flag
+  // and where the wait gave up -- are kept, so that a time-out stays visible to
+  // spark_query_status and later calls return at once until it is read.
+  constexpr size_t kKeep = offsetof(DeviceControl, exit_count);
+  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + kKeep, 0, sizeof(DeviceControl) - kKeep, stream) !=
+      cudaSuccess) {
     cudaGetLastError();
     return SPARK_ECUDA;
   }
@@ -110,7 +140,7 @@ extern "C" SPARK_API int spark_ffn_forward_noalloc(const void* q, const void* K1
   a.theta_out = nullptr;
   a.active_out = nullptr;
   a.workspace = scratch;
-  a.wait_limit_ns = 1000000000ull;
+  a.wait_limit_ns = wait_limit_ns();
   a.never_arrive = 0;
   if (launch_fused(plan, a, stream) != cudaSuccess) {
     cudaGetLastError();

@@ -238,15 +238,23 @@ SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream);
  * returns SPARK_ESCRATCH and enqueues nothing.
  *
  * Set-up: the first call on a device looks up the buffer's device address
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.
+ * (cudaGetSymbolAddress) with that device current and keeps it for the rest of
+ * the process; make that first call before any stream capture.  A
+ * cudaDeviceReset (or any reset of the device's primary context) unmaps the
+ * buffer and leaves that address stale: do not call this entry point on a
+ * device after resetting it.
  *
  * Sharing: all calls on all streams use the same buffer, which keeps the last
- * call's contents.  Each call clears the control block with a cudaMemsetAsync
- * on `stream` before its kernel.  Calls whose work overlaps on the GPU (on
- * different streams, or in graphs replayed concurrently) race on the buffer and
- * give wrong results: order them.  A device-side time-out inside this entry
- * point is not reported by spark_query_status.
+ * call's contents.  Each call clears the buffer's arrival counters with a
+ * cudaMemsetAsync on `stream` before its kernel.  Calls whose work overlaps on
+ * the GPU (on different streams, or in graphs replayed concurrently) race on
+ * the buffer and give wrong results: order them.
+ *
+ * Errors: every device-side wait has the time limit of spark_set_wait_limit_ns.
+ * A wait that runs out leaves `out` undefined and records SPARK_ETIMEOUT in the
+ * buffer; later calls of this entry point then return without computing until
+ * spark_query_status() (on any stream of the device, once the failed call has
+ * completed) reports the error and clears it.
  */
 SPARK_API int spark_ffn_forward_noalloc(const void* q, const void* K1, const void* K2, const void* V,
                                         int d_model, int r, int d_ff, int k, void* out,

@@ -124,8 +124,9 @@ def test_repeatable_and_errors_refused():
                                     out.data_ptr(), st) == -2
 
 
-def test_portable_cluster_size(monkeypatch):
-    """The 8-CTA cluster path (used where 16-CTA clusters are unavailable) keeps parity."""
-    monkeypatch.setenv("SPARK_ATTN_CLUSTER", "8")
-    run_attention(8, 4, 4096, 256, 128, 256, layer=8)
-    run_attention(2, 1, 1000, 128, 64, 100, layer=9)
+def test_portable_cluster_size():
+    """Caches shorter than 512 positions run on 8-CTA clusters (the portable size, also the
+    fallback where 16-CTA clusters are unavailable); parity holds there and at the switch."""
+    run_attention(8, 4, 511, 256, 128, 64, layer=8)
+    run_attention(2, 1, 500, 128, 64, 100, layer=9)
+    run_attention(8, 4, 512, 256, 128, 64, layer=10)

@@ -186,25 +186,6 @@ def test_bounded_wait_times_out_and_recovers():
     run_parity(*TINY, T=4)
 
 
-@pytest.mark.parametrize("cap", ["0", "3"])
-def test_decode_recompute_path_is_bit_identical(cap, monkeypatch):
-    """The one-launch exchange kernel speculates on candidate neurons before theta is known;
-    a CTA whose largest non-candidate score passes theta is recomputed from K1/K2 after the
-    exchange.  Forcing few or no speculation slots must give the same bits, and parity."""
-    monkeypatch.setenv("SPARK_DECODE_IMPL", "exchange")
-    d_model, r, d_ff, k = GEMMA
-    dev, _ = make_layer(d_model, r, d_ff, 1, layer=9)
-    q = dev["q"][0].contiguous()
-    ref = spark.ffn_forward(q, dev["K1"], dev["K2"], dev["V"], k)
-    monkeypatch.setenv("SPARK_DECODE_CAP", cap)
-    forced = spark.ffn_forward(q, dev["K1"], dev["K2"], dev["V"], k)
-    torch.cuda.synchronize()
-    assert spark.query_status() == 0
-    assert torch.equal(forced, ref)
-    monkeypatch.setenv("SPARK_DECODE_CAP", cap)
-    run_parity(*GEMMA, T=1, layer=9)
-
-
 def test_decode_weight_overlap_in_graph_is_bit_identical():
     """Score kernels launched behind the previous call (programmatic dependent launch), in a
     stream and inside a CUDA graph, give the same bits as plain stream order; each call's q
@@ -249,9 +230,3 @@ def test_decode_weight_overlap_in_graph_is_bit_identical():
     finally:
         spark.set_weight_overlap(False)
     assert spark.query_status() == 0
-
-
-def test_decode_exchange_kernel_parity(monkeypatch):
-    """The one-launch exchange kernel (kept as an alternative) stays within parity."""
-    monkeypatch.setenv("SPARK_DECODE_IMPL", "exchange")
-    run_parity(*GEMMA, T=1, layer=50)

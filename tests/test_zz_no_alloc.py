@@ -6,7 +6,7 @@ ahead of time.  For them the library has one entry point whose scratch is a
 fixed buffer inside the library instead of an allocated workspace.  These tests
 call it through the C ABI, twice in a row (the buffer keeps the previous
 call's contents), and compare each result with the allocating entry point's
-under the same tolerance as the other parity tests.  The file name makes
+and with the fp64 oracle's, under the same tolerance as the other parity tests.  The file name makes
 pytest collect it last.
 """
 import ctypes
@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import activation_sparse_transformer_predictor_b200 as spark
 from activation_sparse_transformer_predictor_b200 import _binding
 
@@ -37,14 +38,20 @@ def _noalloc(q, K1, K2, V, k, out):
 def test_noalloc_matches_allocating_entry_point_on_two_calls(shape):
     d_model, r, d_ff, k = shape
     for call, layer in enumerate((40, 41)):
-        dev, _ = make_layer(d_model, r, d_ff, 1, layer=layer)
+        dev, bits = make_layer(d_model, r, d_ff, 1, layer=layer)
         q = dev["q"][0].contiguous()
         ref = spark.ffn_forward(q, dev["K1"], dev["K2"], dev["V"], k)
         out = torch.full_like(ref, float("nan"))
         assert _noalloc(q, dev["K1"], dev["K2"], dev["V"], k, out) == 0, f"call {call}"
         torch.cuda.synchronize()
+        assert spark.query_status() == 0
         assert torch.isfinite(out.float()).all()
+        # against the allocating entry point ...
         assert_outputs_close(bf16_to_f64(out), bf16_to_f64(ref))
+        # ... and against the fp64 oracle (its own active set: neurons that may flip between the
+        # two sit within 1e-4 std of theta and contribute GELU(s) ~ s / 2 ~ 0)
+        orc = oracle.spark_ffn(bits["q"], bits["K1"], bits["K2"], bits["V"], r, k, n_threads=8)["out"]
+        assert_outputs_close(bf16_to_f64(out)[None, :], orc)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
