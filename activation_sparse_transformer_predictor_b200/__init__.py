@@ -18,7 +18,7 @@ from __future__ import annotations
 from . import _binding
 from ._binding import SparkError
 
-__all__ = ["ffn_forward", "ffn_forward_debug", "ffn_decode_stack", "stat_topk_soft_threshold", "query_status", "release_workspace",
+__all__ = ["ffn_forward", "ffn_forward_debug", "ffn_predictor", "ffn_decode_stack", "stat_topk_soft_threshold", "query_status", "release_workspace",
            "topk_quantile", "set_wait_limit_ns", "selftest_wait_timeout", "SparkError"]
 
 
@@ -83,6 +83,24 @@ def ffn_forward_debug(q, K1, K2, V, k: int, stream=None) -> dict:
                                                 theta.data_ptr(), active.data_ptr(), _binding.stream_handle(stream))
     _binding.check("spark_ffn_forward_debug", rc)
     return {"out": out.reshape(q.shape), "x": x, "theta": theta, "active": active}
+
+
+def ffn_predictor(q, K1, out=None, stream=None):
+    """The low-rank predictor alone: x = K1^T q[:r] for each token, fp32 [T, d_ff]."""
+    import torch
+    _require(q, "q", torch.bfloat16, ndim=(1, 2))
+    _require(K1, "K1", torch.bfloat16, ndim=(2,))
+    d_ff, r = K1.shape
+    T = 1 if q.dim() == 1 else q.shape[0]
+    d_model = q.shape[-1]
+    if out is None:
+        out = torch.empty((T, d_ff), dtype=torch.float32, device=q.device)
+    else:
+        _require(out, "out", torch.float32)
+    rc = _binding.lib().spark_ffn_predictor(q.data_ptr(), K1.data_ptr(), T, d_model, r, d_ff, out.data_ptr(),
+                                            _binding.stream_handle(stream))
+    _binding.check("spark_ffn_predictor", rc)
+    return out
 
 
 def ffn_decode_stack(h, layers, k: int, eps: float = 1e-6, h_out=None, debug: bool = False, stream=None):

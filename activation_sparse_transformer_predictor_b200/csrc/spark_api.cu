@@ -283,6 +283,34 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
                           reinterpret_cast<cudaStream_t>(stream), 0);
 }
 
+SPARK_API int spark_ffn_predictor(const void* q, const void* K1, int n_tokens, int d_model, int r, int d_ff,
+                                  float* x_out, spark_stream_t stream_) {
+  if (n_tokens == 0) return SPARK_OK;
+  if (!q || !K1 || !x_out || n_tokens < 0 || d_model < 2 || !(r > 0 && r < d_model) || d_ff < 16)
+    return SPARK_EINVAL;
+  if (r % 8 != 0 || d_model % 8 != 0 || d_ff % 16 != 0) return SPARK_EALIGN;
+  if (!aligned16(q) || !aligned16(K1) || !aligned16(x_out)) return SPARK_EALIGN;
+  const size_t xb = static_cast<size_t>(n_tokens) * d_ff * 4;
+  if (overlaps(x_out, xb, q, static_cast<size_t>(n_tokens) * d_model * 2) ||
+      overlaps(x_out, xb, K1, static_cast<size_t>(d_ff) * r * 2))
+    return SPARK_EINVAL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  void* ws = nullptr;
+  const int wst = get_workspace(dev, stream, predictor_workspace_bytes(n_tokens, d_ff), &ws);
+  if (wst != SPARK_OK) return wst;
+  if (launch_predictor(q, K1, n_tokens, d_model, r, d_ff, x_out, ws, g_wait_limit_ns, di.num_sms, stream) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return SPARK_OK;
+}
+
 SPARK_API int spark_ffn_decode_stack(const float* h_in, float* h_out, const void* const* K1s, const void* const* K2s,
                                      const void* const* Vs, int n_layers, int d_model, int r, int d_ff, int k,
                                      float eps, void* q_dbg, void* out_dbg, spark_stream_t stream_) {

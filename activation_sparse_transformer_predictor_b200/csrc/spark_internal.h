@@ -141,6 +141,9 @@ struct PrefillArgs {
 };
 
 int prefill_splitk(int T, int d_model, int d_ff, int num_sms);
+size_t predictor_workspace_bytes(int T, int d_ff);
+cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, int r, int d_ff, float* x_out,
+                             void* workspace, unsigned long long wait_limit_ns, int num_sms, cudaStream_t stream);
 size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms);
 cudaError_t launch_prefill(const PrefillArgs& args, int num_sms, cudaStream_t stream);
 

@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                 sum += v[j];
                 ++cnt;
               }
-            if (row_ok && n < p.N) {
+            if (row_ok && n < p.N && p.Xt != nullptr) {
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4)
                 xt[(c / 4 + q4) * BM + row] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
@@ -733,6 +733,11 @@ size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 }  // namespace
 
+size_t predictor_workspace_bytes(int T, int d_ff) {
+  const int tiles_n = (d_ff + BN - 1) / BN;
+  return align256(sizeof(DeviceControl)) + align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));
+}
+
 size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms) {
   const int tiles_n = (d_ff + BN - 1) / BN;
   size_t b = align256(sizeof(DeviceControl));
@@ -884,6 +889,46 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+// GEMM 1 alone (the low-rank predictor x = K1^T q[:r] for T tokens), the same
+// kernel and unit choice as in launch_prefill, writing x row-major to x_out
+// instead of the tiled copy GEMM 2 reads; the per-tile moments go to the
+// workspace as usual.
+cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, int r, int d_ff, float* x_out,
+                             void* workspace, unsigned long long wait_limit_ns, int num_sms, cudaStream_t stream) {
+  const int tiles_n = (d_ff + BN - 1) / BN;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const bool a64 = T <= 64;
+  CUtensorMap tq1, tk1;
+  if (!make_tmap(&tq1, q, r, T, static_cast<uint64_t>(d_model) * 2, BK, a64 ? 64 : BM) ||
+      !make_tmap(&tk1, K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, BN))
+    return cudaErrorInvalidValue;
+  GemmParams g{};
+  g.ctl = reinterpret_cast<DeviceControl*>(ws);
+  g.wait_limit_ns = wait_limit_ns;
+  g.X = x_out;
+  g.Xt = nullptr;
+  g.xt_tiles_n = tiles_n;
+  g.moments = reinterpret_cast<float2*>(ws + align256(sizeof(DeviceControl)));
+  g.mom_stride = tiles_n;
+  g.M = T;
+  g.N = d_ff;
+  g.K = r;
+  g.tiles_m = (T + BM - 1) / BM;
+  g.tiles_n = tiles_n;
+  g.nkb = (r + BK - 1) / BK;
+  g.split_k = 1;
+  g.kb_per_split = g.nkb;
+  g.units = g.tiles_m * g.tiles_n;
+  const int wide_units = g.tiles_m * ((d_ff + 2 * BN - 1) / (2 * BN));
+  if (wide_units >= num_sms) {
+    g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
+    g.units = wide_units;
+    return launch_gemm<kEpiPredictor, false, false, 4, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  }
+  if (a64) return launch_gemm<kEpiPredictor, false, false, 8, false, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  return launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
 }
 
 }  // namespace spark

@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill / stat-topk extra lines")
-    ap.add_argument("--case", default=None, choices=["decode", "prefill", "topk", "attention"],
+    ap.add_argument("--case", default=None, choices=["decode", "prefill", "predictor", "topk", "attention"],
                     help="profiling mode: run only this workload, plain launches (no graph), print per-call time")
     ap.add_argument("--tokens", type=int, default=256, help="--case prefill: tokens per call")
     return ap.parse_args()
@@ -341,6 +341,13 @@ def run_case(args):
         fn = lambda i: spark.attention_decode(caches[i % 4]["q"], caches[i % 4]["K"], caches[i % 4]["V"], 128, 256,
                                               scale=1.0 / _m.sqrt(256), out=aout)
         unit = "attention 8/4 heads x 4096 positions"
+    elif args.case == "predictor":
+        w = synthetic.ffn_layer(D_MODEL, R, D_FF)
+        k1s = [w["K1"].to(dev)] + [w["K1"].to(dev).clone() for _ in range(3)]
+        q = synthetic.tokens(args.tokens, D_MODEL, layer=1).to(dev)
+        xo = torch.empty((args.tokens, D_FF), dtype=torch.float32, device=dev)
+        fn = lambda i: spark.ffn_predictor(q, k1s[i % len(k1s)], out=xo)
+        unit = f"predictor GEMM, T={args.tokens}"
     elif args.case == "topk":
         rows, d, k = 8 * 4096, 4096, 256
         x = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
@@ -465,7 +472,7 @@ def main():
             "note": "score kernel launched after the previous call completes"},
     }
     if not args.no_extra:
-        also.update(extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs))
+        also.update(extra_workloads(spark, synthetic, torch, dev, base, copies, world, args, hbm_gbs))
 
     if rank == 0:
         cpu = oracle_baseline(args.cpu_seconds) if world == 1 or rank == 0 else None
@@ -500,11 +507,15 @@ def main():
         dist.destroy_process_group()
 
 
-def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
+def extra_workloads(spark, synthetic, torch, dev, base, copies, world, args, hbm_gbs):
     from activation_sparse_transformer_predictor_b200 import _binding
     L = _binding.lib()
     bf16_tflops = peaks()[1]  # burst: each prefill call is timed by itself
     res = {}
+    # mean number of active neurons per token on these inputs (for the method's own FLOP count)
+    qm = synthetic.tokens(64, D_MODEL, layer=1).to(dev)
+    m_mean = float(spark.ffn_forward_debug(qm, base["K1"], base["K2"], base["V"], K)["active"].sum().item()) / 64
+    del qm
     # batched prefill, T = 256 and T = 4096 (one layer; whole-call throughput: predictor GEMM, theta,
     # gate GEMM, output GEMM and split-K reduce)
     for T, reps in ((16, 80), (64, 80), (256, 40), (1024, 16), (4096, 8)):
@@ -520,13 +531,19 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
 
         ms, n = time_graph([pre] * 4, reps, args.warmup, world)
         ms = max_over_ranks(ms, world)
-        flops = 2.0 * T * D_FF * (R + (D_MODEL - R) + 2 * D_MODEL)  # executed: predictor + gate (a) + 2-part output
+        # the method's own work: predictor 2 r d_ff, then 2 (d - r) + 2 d per active neuron
+        aflops = T * (2.0 * R * D_FF + 2.0 * m_mean * (2 * D_MODEL - R))
+        # what the kernels execute: predictor + gate (a) + two-part output, dense over the tile union
+        xflops = 2.0 * T * D_FF * (R + (D_MODEL - R) + 2 * D_MODEL)
         # algorithmic bytes: K1 once, the expected union of the tokens' active K2 / V rows, q and out
         union = D_FF * (1.0 - (1.0 - K / D_FF) ** T)
         abytes = D_FF * R * 2 + union * ((D_MODEL - R) + D_MODEL) * 2 + 2 * T * D_MODEL * 2
         res[f"prefill_T{T}"] = {"tokens_per_s": whole_job_rate(T, ms, world), "ms_per_call": ms,
-                                "executed_tflops": flops / (ms * 1e-3) / 1e12,
-                                "frac_of_bf16_peak": flops / (ms * 1e-3) / 1e12 / bf16_tflops,
+                                "algorithmic_tflops": aflops / (ms * 1e-3) / 1e12,
+                                "frac_of_bf16_peak": aflops / (ms * 1e-3) / 1e12 / bf16_tflops,
+                                "executed_tflops": xflops / (ms * 1e-3) / 1e12,
+                                "executed_frac_of_bf16_peak": xflops / (ms * 1e-3) / 1e12 / bf16_tflops,
+                                "mean_active_per_token": m_mean,
                                 "algorithmic_bytes": abytes,
                                 "frac_of_hbm_peak": abytes / (ms * 1e-3) / 1e9 / hbm_gbs,
                                 "note": "one layer; whole call (three GEMMs, plus the threshold and split-K reduce "
@@ -534,6 +551,27 @@ def extra_workloads(spark, synthetic, torch, dev, base, world, args, hbm_gbs):
                                         "dense 128-token tiles (the union of per-token active sets covers "
                                         "~every neuron); per-kernel live spans are in the prefill profile"}
         del q, out
+    # the predictor GEMM alone (spark_ffn_predictor: x = K1^T q[:r]), cycling over the 16 K1 copies
+    for T in (256, 1024, 4096):
+        q = synthetic.tokens(T, D_MODEL, layer=1).to(dev)
+        xo = torch.empty((T, D_FF), dtype=torch.float32, device=dev)
+
+        def pred(c, q=q, xo=xo, T=T):
+            def f():
+                rc = L.spark_ffn_predictor(q.data_ptr(), c["K1"].data_ptr(), T, D_MODEL, R, D_FF, xo.data_ptr(),
+                                           _binding.stream_handle())
+                if rc != 0:
+                    raise _binding.SparkError("spark_ffn_predictor", rc)
+            return f
+
+        ms, n = time_graph([pred(c) for c in copies], 16 * max(1, 64 // (T // 256)), args.warmup, world)
+        ms = max_over_ranks(ms, world)
+        tf = 2.0 * T * R * D_FF / (ms * 1e-3) / 1e12
+        res[f"predictor_gemm_T{T}"] = {"ms_per_call": ms, "tflops": tf, "frac_of_bf16_peak": tf / bf16_tflops,
+                                       "peak": bf16_tflops, "peak_kind": "measured bf16 burst",
+                                       "note": "GEMM 1 alone (tcgen05, fp32 x stored row-major), 2 T r d_ff flops "
+                                               "per call, 16 K1 copies cycled (340 MB > L2)"}
+        del q, xo
     # 26-layer decode stack (Gemma-2-2B depth), one token, residual + RMSNorm between layers
     import ctypes
     n_layers = 26

@@ -102,6 +102,18 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
                                       spark_stream_t stream);
 
 /*
+ * The low-rank predictor alone ("Spark FFN": x = K1^T q[:r]) for n_tokens
+ * tokens: x_out[t][i] = <K1[i,:], q[t][:r]>, fp32 [n_tokens][d_ff], 16-byte
+ * aligned, not overlapping q or K1.  The same tensor-core GEMM (bf16 operands,
+ * fp32 accumulation) as the predictor stage of batched prefill.  q is bf16
+ * [n_tokens][d_model] (only q[:, :r] is read), K1 bf16 [d_ff][r].  Requires
+ * 0 < r < d_model, r and d_model multiples of 8, d_ff a multiple of 16
+ * (else SPARK_EALIGN).  n_tokens == 0 is a no-op.
+ */
+SPARK_API int spark_ffn_predictor(const void* q, const void* K1, int n_tokens, int d_model, int r, int d_ff,
+                                  float* x_out, spark_stream_t stream);
+
+/*
  * A decoder stack of Spark FFN layers for one token (decode).  Between layers it
  * applies the pre-norm residual of a Gemma-style stack (the notes place Spark FFN
  * inside a Gemma-2 model but do not spell this out; it is how the layers chain):

@@ -79,3 +79,12 @@ def test_argument_checks_before_any_device_work(L):
     assert t(fake, 0, 100, 10, fake, null) == 0  # no rows: no-op
     assert t(fake, 4, 100, 10, vp((1 << 20) + 16), null) == EINVAL  # partial overlap
     assert t(vp((1 << 20) + 2), 4, 100, 10, vp(1 << 30), null) == EALIGN  # not 4-byte aligned
+    p = L.spark_ffn_predictor
+    assert p(fake, fake, 0, 64, 32, 256, vp(1 << 30), null) == 0  # no tokens: no-op
+    assert p(null, fake, 2, 64, 32, 256, vp(1 << 30), null) == EINVAL
+    assert p(fake, fake, -1, 64, 32, 256, vp(1 << 30), null) == EINVAL
+    assert p(fake, fake, 2, 64, 64, 256, vp(1 << 30), null) == EINVAL  # r == d_model
+    assert p(fake, fake, 2, 64, 32, 264, vp(1 << 30), null) == EALIGN  # d_ff % 16
+    assert p(fake, fake, 2, 64, 36, 256, vp(1 << 30), null) == EALIGN  # r % 8
+    assert p(fake, fake, 2, 64, 32, 256, vp((1 << 30) + 4), null) == EALIGN  # x_out alignment
+    assert p(fake, fake, 2, 64, 32, 256, vp((1 << 20) + 64), null) == EINVAL  # x_out overlapping q
