@@ -99,6 +99,8 @@ DECODE_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/ffn_decode_
                   "activation_sparse_transformer_predictor_b200/csrc/spark_device.cuh"]
 TOPK_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/stat_topk.cu",
                 "activation_sparse_transformer_predictor_b200/csrc/spark_device.cuh"]
+PRED_SOURCES = ["activation_sparse_transformer_predictor_b200/csrc/umma_gemm.cu",
+                "activation_sparse_transformer_predictor_b200/csrc/spark_device.cuh"]
 
 
 class ClockSampler:
@@ -569,6 +571,8 @@ def extra_workloads(spark, synthetic, torch, dev, base, copies, world, args, hbm
         tf = 2.0 * T * R * D_FF / (ms * 1e-3) / 1e12
         res[f"predictor_gemm_T{T}"] = {"ms_per_call": ms, "tflops": tf, "frac_of_bf16_peak": tf / bf16_tflops,
                                        "peak": bf16_tflops, "peak_kind": "measured bf16 burst",
+                                       "traffic": profile_traffic("umma_gemm_predictor_gemma_T256.txt", PRED_SOURCES)
+                                       if T == 256 else None,
                                        "note": "GEMM 1 alone (tcgen05, fp32 x stored row-major), 2 T r d_ff flops "
                                                "per call, 16 K1 copies cycled (340 MB > L2)"}
         del q, xo
