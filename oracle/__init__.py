@@ -68,6 +68,10 @@ def _load():
         lib.oracle_stat_topk.argtypes = [ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_long,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_stat_topk_causal.restype = ctypes.c_int
+        lib.oracle_stat_topk_causal.argtypes = [ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_long,
+                                                ctypes.c_long, ctypes.c_long, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_int]
         lib.oracle_spark_ffn.restype = ctypes.c_int
         lib.oracle_spark_ffn.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_long] * 5 + [
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -151,6 +155,23 @@ def stat_topk(x: np.ndarray, k: int, n_threads: int = 1):
     if rc != 0:
         raise ValueError(f"oracle_stat_topk: invalid arguments (d={d}, k={k})")
     return out, th, mu, sd
+
+
+def stat_topk_causal(x: np.ndarray, k: int, n_q: int, offset: int = 0, n_threads: int = 1):
+    """Statistical top-k + soft threshold on causally masked fp32 rows [rows, d]: row i sees its
+    first min(d, offset + i % n_q + 1) entries.  Returns (out fp64 [rows, d], theta [rows];
+    theta = -inf on rows whose visible entries number at most k, which pass through unshifted)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim == 1:
+        x = x[None, :]
+    rows, d = x.shape
+    out = np.empty((rows, d), dtype=np.float64)
+    th = np.empty(rows, dtype=np.float64)
+    rc = _load().oracle_stat_topk_causal(_ptr(x), rows, d, int(k), int(n_q), int(offset), _ptr(out), _ptr(th),
+                                         int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_stat_topk_causal: invalid arguments (d={d}, k={k}, n_q={n_q}, offset={offset})")
+    return out, th
 
 
 def spark_ffn(q_bits, K1_bits, K2_bits, V_bits, r: int, k: int, gelu_kind: int = GELU_TANH,

@@ -155,6 +155,52 @@ int oracle_stat_topk(const float *x, long rows, long d, long k, double *out,
 }
 
 /*
+ * Statistical top-k with soft threshold on causally masked score rows (the
+ * attention-shaped case of "Statistical Top-k" under a causal mask; "Spark
+ * Attention": each token attends to at most k_attn tokens, so the work is
+ * min{k_attn, n_ctx} per query).
+ *   Row i is query number i mod n_q of its head, at position
+ *   pos = offset + (i mod n_q); it sees keys 0..pos, i.e. the first
+ *   n = min(d, pos + 1) entries of the row; the rest are masked.
+ *   If k < n: theta = mean + std * Q(1 - k/n) over the n visible entries
+ *     (population std), out[j] = max(x[j] - theta, 0) for j < n.
+ *   If k >= n: every visible entry is kept (the threshold formula has no
+ *     finite value there, Q(1 - k/n) = -inf): theta = -inf and out[j] = x[j]
+ *     for j < n (the scores pass through unshifted).
+ *   Masked entries (j >= n) are 0 in both cases.
+ * theta_out optional (NULL to skip).  Returns 0, or -1 unless k >= 1, n_q >= 1,
+ * offset >= 0, d >= 1, rows >= 0.
+ */
+int oracle_stat_topk_causal(const float *x, long rows, long d, long k, long n_q, long offset, double *out,
+                            double *theta_out, int n_threads)
+{
+    if (k < 1 || n_q < 1 || offset < 0 || d < 1 || rows < 0) return -1;
+    if (n_threads < 1) n_threads = 1;
+#pragma omp parallel for schedule(static) num_threads(n_threads)
+    for (long row = 0; row < rows; ++row) {
+        const long pos = offset + row % n_q;
+        const long n = pos + 1 < d ? pos + 1 : d;
+        double *xr = (double *)malloc(sizeof(double) * (size_t)n);
+        for (long j = 0; j < n; ++j) xr[j] = (double)x[row * d + j];
+        double theta = -INFINITY;
+        if (k < n) {
+            double mean, sd;
+            theta = oracle_theta(xr, n, k, &mean, &sd);
+            for (long j = 0; j < n; ++j) {
+                double s = xr[j] - theta;
+                out[row * d + j] = s > 0.0 ? s : 0.0;
+            }
+        } else {
+            for (long j = 0; j < n; ++j) out[row * d + j] = xr[j];
+        }
+        for (long j = n; j < d; ++j) out[row * d + j] = 0.0;
+        if (theta_out) theta_out[row] = theta;
+        free(xr);
+    }
+    return 0;
+}
+
+/*
  * Spark FFN forward over T tokens ("Spark FFN" in 关键设计):
  *   x_i   = sum_{j<r} K1[i][j] q[j]                       (predictor, K1 is d_ff x r)
  *   theta = mean(x) + std(x) Q(1 - k/d_ff)                 (statistical top-k)

@@ -48,6 +48,19 @@ ATTN_MUTATIONS = {
 }
 
 
+# Mistakes planted in the causal statistical top-k; the causal pins must catch each.
+CAUSAL_MUTATIONS = {
+    "causal_visible_count_off_by_one": ("const long n = pos + 1 < d ? pos + 1 : d;", "const long n = pos < d ? pos : d;"),
+    "causal_heads_not_wrapped": ("const long pos = offset + row % n_q;", "const long pos = offset + row;"),
+    "causal_offset_ignored": ("const long pos = offset + row % n_q;", "const long pos = row % n_q;"),
+    "causal_masked_not_zeroed": ("for (long j = n; j < d; ++j) out[row * d + j] = 0.0;",
+                                 "for (long j = n; j < d; ++j) out[row * d + j] = (double)x[row * d + j];"),
+    "causal_select_all_zeroed": ("for (long j = 0; j < n; ++j) out[row * d + j] = xr[j];",
+                                 "for (long j = 0; j < n; ++j) out[row * d + j] = 0.0;"),
+    "causal_select_all_boundary": ("        if (k < n) {\n            double mean, sd;", "        if (k <= n) {\n            double mean, sd;"),
+}
+
+
 def _pins_fail_on(old, new, pin_file, tmp_path):
     src = open(SRC).read()
     assert src.count(old) == 1, "mutation anchor not found exactly once"
@@ -85,3 +98,10 @@ def test_pins_catch_planted_mistake(name, tmp_path):
                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                           env=env, cwd=ROOT, capture_output=True, text=True, timeout=300)
     assert proc.returncode != 0, f"pins did not catch mutation {name}:\n{proc.stdout[-2000:]}"
+
+
+@pytest.mark.parametrize("name", sorted(CAUSAL_MUTATIONS))
+def test_causal_pins_catch_planted_mistake(name, tmp_path):
+    old, new = CAUSAL_MUTATIONS[name]
+    caught, log = _pins_fail_on(old, new, "test_oracle_causal_pins.py", tmp_path)
+    assert caught, f"causal pins did not catch mutation {name}:\n{log}"
