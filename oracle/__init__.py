@@ -68,6 +68,13 @@ def _load():
         lib.oracle_stat_topk.argtypes = [ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_long,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_int]
+        lib.oracle_stat_topk_huber.restype = ctypes.c_int
+        lib.oracle_stat_topk_huber.argtypes = [ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_long,
+                                               ctypes.c_double, ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_stat_topk_huber_backward.restype = ctypes.c_int
+        lib.oracle_stat_topk_huber_backward.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_long,
+                                                        ctypes.c_long, ctypes.c_long, ctypes.c_double,
+                                                        ctypes.c_void_p]
         lib.oracle_stat_topk_causal.restype = ctypes.c_int
         lib.oracle_stat_topk_causal.argtypes = [ctypes.c_void_p, ctypes.c_long, ctypes.c_long, ctypes.c_long,
                                                 ctypes.c_long, ctypes.c_long, ctypes.c_void_p, ctypes.c_void_p,
@@ -155,6 +162,35 @@ def stat_topk(x: np.ndarray, k: int, n_threads: int = 1):
     if rc != 0:
         raise ValueError(f"oracle_stat_topk: invalid arguments (d={d}, k={k})")
     return out, th, mu, sd
+
+
+def stat_topk_huber(x: np.ndarray, k: int, delta: float):
+    """Huber-smoothed statistical top-k on fp64 rows [rows, d]: out = rho_delta(x - theta(x)).
+    Returns (out [rows, d], theta [rows])."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    if x.ndim == 1:
+        x = x[None, :]
+    rows, d = x.shape
+    out = np.empty((rows, d), dtype=np.float64)
+    th = np.empty(rows, dtype=np.float64)
+    if _load().oracle_stat_topk_huber(_ptr(x), rows, d, int(k), float(delta), _ptr(out), _ptr(th)) != 0:
+        raise ValueError(f"oracle_stat_topk_huber: invalid arguments (d={d}, k={k}, delta={delta})")
+    return out, th
+
+
+def stat_topk_huber_backward(x: np.ndarray, g: np.ndarray, k: int, delta: float) -> np.ndarray:
+    """dL/dx of the Huber-smoothed statistical top-k for upstream gradient g (both fp64 [rows, d])."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    if x.ndim == 1:
+        x, g = x[None, :], g[None, :]
+    if g.shape != x.shape:
+        raise ValueError("stat_topk_huber_backward: x and g differ in shape")
+    rows, d = x.shape
+    dx = np.empty((rows, d), dtype=np.float64)
+    if _load().oracle_stat_topk_huber_backward(_ptr(x), _ptr(g), rows, d, int(k), float(delta), _ptr(dx)) != 0:
+        raise ValueError(f"oracle_stat_topk_huber_backward: invalid arguments (d={d}, k={k}, delta={delta})")
+    return dx
 
 
 def stat_topk_causal(x: np.ndarray, k: int, n_q: int, offset: int = 0, n_threads: int = 1):

@@ -155,6 +155,84 @@ int oracle_stat_topk(const float *x, long rows, long d, long k, double *out,
 }
 
 /*
+ * Huber-smoothed statistical top-k ("Statistical Top-k", Theorem 3.2: after
+ * smoothing with a Huber function the operator is continuously
+ * differentiable).  Reading: the kink of Soft-Threshold, max{z, 0} at z = 0,
+ * is replaced by the Huber-smoothed ramp of width delta >= 0
+ *   rho(z) = 0                 for z <= 0
+ *          = z^2 / (2 delta)   for 0 < z < delta
+ *          = z - delta / 2     for z >= delta
+ * (delta = 0: rho(z) = max{z, 0}, the plain operator), with z = x - theta(x),
+ * theta(x) = mean(x) + std(x) Q(1 - k/d), population std, as everywhere here.
+ */
+static double huber_ramp(double z, double delta)
+{
+    if (z <= 0.0) return 0.0;
+    if (z < delta) return z * z / (2.0 * delta);
+    return z - 0.5 * delta;
+}
+
+/* rho'(z): 0, z / delta, 1 on the three pieces (0 at the kink when delta = 0). */
+static double huber_ramp_slope(double z, double delta)
+{
+    if (z <= 0.0) return 0.0;
+    if (z < delta) return z / delta;
+    return 1.0;
+}
+
+/* Forward on fp64 rows: out = rho(x - theta(x)).  Returns 0, or -1 unless
+ * 0 < k < d and delta >= 0. */
+int oracle_stat_topk_huber(const double *x, long rows, long d, long k, double delta, double *out,
+                           double *theta_out)
+{
+    if (!(k > 0 && k < d) || rows < 0 || !(delta >= 0.0)) return -1;
+    for (long row = 0; row < rows; ++row) {
+        const double *xr = x + row * d;
+        double mean, sd;
+        double theta = oracle_theta(xr, d, k, &mean, &sd);
+        for (long i = 0; i < d; ++i) out[row * d + i] = huber_ramp(xr[i] - theta, delta);
+        if (theta_out) theta_out[row] = theta;
+    }
+    return 0;
+}
+
+/*
+ * Backward (vector-Jacobian product) of the forward above for an upstream
+ * gradient g = dL/dout.  By the chain rule, with w_i = g_i rho'(z_i) and
+ * W = sum_i w_i,
+ *   dL/dx_j = w_j - W dtheta/dx_j,
+ *   dtheta/dx_j = 1/d + Q(1 - k/d) (x_j - mean) / (d std)
+ * (d mean/dx_j = 1/d; d std/dx_j = (x_j - mean) / (d std)).  A row with zero
+ * spread has every z = 0, so w = 0 and the result is 0 (the std term is not
+ * evaluated there).  Returns 0, or -1 on invalid arguments.
+ */
+int oracle_stat_topk_huber_backward(const double *x, const double *g, long rows, long d, long k, double delta,
+                                    double *grad_x)
+{
+    if (!(k > 0 && k < d) || rows < 0 || !(delta >= 0.0)) return -1;
+    const double Q = oracle_topk_quantile((double)k, (double)d);
+    double *w = (double *)malloc(sizeof(double) * (size_t)d);
+    for (long row = 0; row < rows; ++row) {
+        const double *xr = x + row * d;
+        const double *gr = g + row * d;
+        double mean, sd;
+        double theta = oracle_theta(xr, d, k, &mean, &sd);
+        double W = 0.0;
+        for (long i = 0; i < d; ++i) {
+            w[i] = gr[i] * huber_ramp_slope(xr[i] - theta, delta);
+            W += w[i];
+        }
+        for (long j = 0; j < d; ++j) {
+            double dtheta = 1.0 / (double)d;
+            if (sd > 0.0) dtheta += Q * (xr[j] - mean) / ((double)d * sd);
+            grad_x[row * d + j] = w[j] - W * dtheta;
+        }
+    }
+    free(w);
+    return 0;
+}
+
+/*
  * Statistical top-k with soft threshold on causally masked score rows (the
  * attention-shaped case of "Statistical Top-k" under a causal mask; "Spark
  * Attention": each token attends to at most k_attn tokens, so the work is

@@ -61,6 +61,18 @@ CAUSAL_MUTATIONS = {
 }
 
 
+# Mistakes planted in the Huber-smoothed forward and its backward; the Huber pins must catch each.
+HUBER_MUTATIONS = {
+    "huber_backward_drops_theta": ("grad_x[row * d + j] = w[j] - W * dtheta;", "grad_x[row * d + j] = w[j];"),
+    "huber_backward_theta_sign": ("grad_x[row * d + j] = w[j] - W * dtheta;", "grad_x[row * d + j] = w[j] + W * dtheta;"),
+    "huber_backward_drops_std_term": ("if (sd > 0.0) dtheta += Q * (xr[j] - mean) / ((double)d * sd);",
+                                      "if (sd > 0.0) dtheta += 0.0;"),
+    "huber_middle_slope": ("if (z < delta) return z / delta;", "if (z < delta) return z / (2.0 * delta);"),
+    "huber_forward_offset": ("return z - 0.5 * delta;", "return z - delta;"),
+    "huber_forward_square": ("if (z < delta) return z * z / (2.0 * delta);", "if (z < delta) return z * z / delta;"),
+}
+
+
 def _pins_fail_on(old, new, pin_file, tmp_path):
     src = open(SRC).read()
     assert src.count(old) == 1, "mutation anchor not found exactly once"
@@ -105,3 +117,10 @@ def test_causal_pins_catch_planted_mistake(name, tmp_path):
     old, new = CAUSAL_MUTATIONS[name]
     caught, log = _pins_fail_on(old, new, "test_oracle_causal_pins.py", tmp_path)
     assert caught, f"causal pins did not catch mutation {name}:\n{log}"
+
+
+@pytest.mark.parametrize("name", sorted(HUBER_MUTATIONS))
+def test_huber_pins_catch_planted_mistake(name, tmp_path):
+    old, new = HUBER_MUTATIONS[name]
+    caught, log = _pins_fail_on(old, new, "test_oracle_huber_pins.py", tmp_path)
+    assert caught, f"Huber pins did not catch mutation {name}:\n{log}"
