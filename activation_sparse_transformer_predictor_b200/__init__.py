@@ -18,7 +18,8 @@ from __future__ import annotations
 from . import _binding
 from ._binding import SparkError
 
-__all__ = ["ffn_forward", "ffn_forward_debug", "ffn_predictor", "ffn_decode_stack", "stat_topk_soft_threshold", "query_status", "release_workspace",
+__all__ = ["ffn_forward", "ffn_forward_debug", "ffn_predictor", "ffn_decode_stack", "stat_topk_soft_threshold",
+           "stat_topk_soft_threshold_causal", "stat_topk_huber", "stat_topk_huber_backward", "query_status", "release_workspace",
            "topk_quantile", "set_wait_limit_ns", "selftest_wait_timeout", "SparkError"]
 
 
@@ -144,6 +145,64 @@ def stat_topk_soft_threshold(x, k: int, out=None, stream=None):
                                                  _binding.stream_handle(stream))
     _binding.check("stat_topk_soft_threshold", rc)
     return out
+
+
+def stat_topk_soft_threshold_causal(x, k: int, n_q: int | None = None, offset: int = 0, out=None, theta=None,
+                                    stream=None):
+    """Statistical top-k with soft threshold on causally masked fp32 rows [rows, d]: row r sees its first
+    min(d, offset + r % n_q + 1) entries (n_q defaults to d: square causal scores); rows seeing at most k
+    entries keep them all (theta = -inf).  Returns out, or (out, theta) when theta is a tensor to fill."""
+    import torch
+    _require(x, "x", torch.float32)
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    n_q = d if n_q is None else int(n_q)
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _require(out, "out", torch.float32)
+    if theta is not None:
+        _require(theta, "theta", torch.float32)
+    rc = _binding.lib().stat_topk_soft_threshold_causal(x.data_ptr(), rows, d, int(k), n_q, int(offset),
+                                                        out.data_ptr(), _binding.ptr(theta),
+                                                        _binding.stream_handle(stream))
+    _binding.check("stat_topk_soft_threshold_causal", rc)
+    return out if theta is None else (out, theta)
+
+
+def stat_topk_huber(x, k: int, delta: float, out=None, stream=None):
+    """Huber-smoothed statistical top-k on fp32 rows [rows, d]: out = rho_delta(x - theta(x))."""
+    import torch
+    _require(x, "x", torch.float32)
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    if out is None:
+        out = torch.empty_like(x)
+    else:
+        _require(out, "out", torch.float32)
+    rc = _binding.lib().stat_topk_huber(x.data_ptr(), rows, d, int(k), float(delta), out.data_ptr(),
+                                        _binding.stream_handle(stream))
+    _binding.check("stat_topk_huber", rc)
+    return out
+
+
+def stat_topk_huber_backward(x, grad_out, k: int, delta: float, grad_x=None, stream=None):
+    """Gradient of sum(grad_out * stat_topk_huber(x)) with respect to x (fp32 [rows, d])."""
+    import torch
+    _require(x, "x", torch.float32)
+    _require(grad_out, "grad_out", torch.float32)
+    if grad_out.shape != x.shape:
+        raise ValueError("stat_topk_huber_backward: x and grad_out differ in shape")
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    if grad_x is None:
+        grad_x = torch.empty_like(x)
+    else:
+        _require(grad_x, "grad_x", torch.float32)
+    rc = _binding.lib().stat_topk_huber_backward(x.data_ptr(), grad_out.data_ptr(), rows, d, int(k), float(delta),
+                                                 grad_x.data_ptr(), _binding.stream_handle(stream))
+    _binding.check("stat_topk_huber_backward", rc)
+    return grad_x
 
 
 def query_status(stream=None) -> int:

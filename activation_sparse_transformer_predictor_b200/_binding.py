@@ -24,7 +24,8 @@ EXPORTS = ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_d
            "spark_query_status", "spark_release_workspace", "spark_status_string", "spark_topk_quantile",
            "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc",
            "spark_ffn_decode_stack", "spark_set_weight_overlap", "spark_attention_decode",
-           "spark_attention_decode_debug", "spark_ffn_predictor")
+           "spark_attention_decode_debug", "spark_ffn_predictor", "stat_topk_soft_threshold_causal",
+           "stat_topk_huber", "stat_topk_huber_backward")
 
 _lock = threading.Lock()
 _lib = None
@@ -67,11 +68,15 @@ def lib() -> ctypes.CDLL:
         L.spark_ffn_forward_noalloc.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
         L.spark_ffn_decode_stack.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ctypes.c_float, vp, vp, vp]
         L.spark_ffn_predictor.argtypes = [vp, vp, ci, ci, ci, ci, vp, vp]
+        L.stat_topk_soft_threshold_causal.argtypes = [vp, ci, ci, ci, ci, ci, vp, vp, vp]
+        L.stat_topk_huber.argtypes = [vp, ci, ci, ci, ctypes.c_float, vp, vp]
+        L.stat_topk_huber_backward.argtypes = [vp, vp, ci, ci, ci, ctypes.c_float, vp, vp]
         for name in ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_debug",
                      "stat_topk_soft_threshold", "spark_query_status", "spark_release_workspace",
                      "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc",
                      "spark_ffn_decode_stack", "spark_set_weight_overlap", "spark_attention_decode",
-                     "spark_attention_decode_debug", "spark_ffn_predictor"):
+                     "spark_attention_decode_debug", "spark_ffn_predictor", "stat_topk_soft_threshold_causal",
+                     "stat_topk_huber", "stat_topk_huber_backward"):
             getattr(L, name).restype = ci
         _lib = L
         return L

@@ -443,6 +443,78 @@ SPARK_API int stat_topk_soft_threshold(const float* x, int rows, int d, int k, f
   return SPARK_OK;
 }
 
+SPARK_API int stat_topk_huber(const float* x, int rows, int d, int k, float delta, float* out, spark_stream_t stream) {
+  if (rows == 0) return SPARK_OK;
+  if (!x || !out || rows < 0 || d < 2 || !(k > 0 && k < d) || !(delta >= 0.f) || !std::isfinite(delta))
+    return SPARK_EINVAL;
+  const size_t bytes = static_cast<size_t>(rows) * d * sizeof(float);
+  if (x != out && overlaps(x, bytes, out, bytes)) return SPARK_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 3u) return SPARK_EALIGN;
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d)));
+  if (launch_stat_topk_huber(x, out, rows, d, Q, delta, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return SPARK_OK;
+}
+
+SPARK_API int stat_topk_huber_backward(const float* x, const float* grad_out, int rows, int d, int k, float delta,
+                                       float* grad_x, spark_stream_t stream) {
+  if (rows == 0) return SPARK_OK;
+  if (!x || !grad_out || !grad_x || rows < 0 || d < 2 || !(k > 0 && k < d) || !(delta >= 0.f) ||
+      !std::isfinite(delta))
+    return SPARK_EINVAL;
+  const size_t bytes = static_cast<size_t>(rows) * d * sizeof(float);
+  // grad_x may be x or grad_out itself (in place); any other overlap is refused
+  if ((grad_x != x && overlaps(grad_x, bytes, x, bytes)) ||
+      (grad_x != grad_out && overlaps(grad_x, bytes, grad_out, bytes)))
+    return SPARK_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(grad_out) | reinterpret_cast<uintptr_t>(grad_x)) &
+      3u)
+    return SPARK_EALIGN;
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  const float Q = static_cast<float>(upper_tail_quantile(static_cast<double>(k) / static_cast<double>(d)));
+  if (launch_stat_topk_huber_backward(x, grad_out, grad_x, rows, d, Q, delta,
+                                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return SPARK_OK;
+}
+
+SPARK_API int stat_topk_soft_threshold_causal(const float* x, int rows, int d, int k, int n_q, int offset,
+                                              float* out, float* theta_out, spark_stream_t stream) {
+  if (rows == 0) return SPARK_OK;
+  if (!x || !out || rows < 0 || d < 1 || k < 1 || n_q < 1 || offset < 0) return SPARK_EINVAL;
+  const size_t bytes = static_cast<size_t>(rows) * d * sizeof(float);
+  if (x != out && overlaps(x, bytes, out, bytes)) return SPARK_EINVAL;
+  if (theta_out != nullptr && (overlaps(theta_out, static_cast<size_t>(rows) * 4, x, bytes) ||
+                               overlaps(theta_out, static_cast<size_t>(rows) * 4, out, bytes)))
+    return SPARK_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(theta_out)) & 3u)
+    return SPARK_EALIGN;
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int st = device_info(dev, &di);
+  if (st != SPARK_OK) return st;
+  if (launch_stat_topk_causal(x, out, rows, d, k, n_q, offset, theta_out, reinterpret_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return SPARK_OK;
+}
+
 SPARK_API int spark_query_status(spark_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (cudaStreamSynchronize(stream) != cudaSuccess) {

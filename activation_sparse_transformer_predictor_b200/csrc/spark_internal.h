@@ -21,6 +21,12 @@ int noalloc_take_status(int dev);
 
 // ---------------------------------------------------------------- stat top-k
 cudaError_t launch_stat_topk(const float* x, float* out, int rows, int d, float Q, cudaStream_t stream);
+cudaError_t launch_stat_topk_huber(const float* x, float* out, int rows, int d, float Q, float delta,
+                                   cudaStream_t stream);
+cudaError_t launch_stat_topk_huber_backward(const float* x, const float* g, float* gx, int rows, int d, float Q,
+                                            float delta, cudaStream_t stream);
+cudaError_t launch_stat_topk_causal(const float* x, float* out, int rows, int d, int k, int n_q, int offset,
+                                    float* theta_out, cudaStream_t stream);
 
 // ---------------------------------------------------------------- fused decode / small-batch FFN
 constexpr int kFusedMaxTokens = 4;     // tokens per launch of the fused kernel

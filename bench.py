@@ -51,7 +51,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill / stat-topk extra lines")
-    ap.add_argument("--case", default=None, choices=["decode", "prefill", "predictor", "topk", "attention"],
+    ap.add_argument("--case", default=None, choices=["decode", "prefill", "predictor", "topk", "topk_causal",
+                                                     "huber_bwd", "attention"],
                     help="profiling mode: run only this workload, plain launches (no graph), print per-call time")
     ap.add_argument("--tokens", type=int, default=256, help="--case prefill: tokens per call")
     return ap.parse_args()
@@ -350,6 +351,19 @@ def run_case(args):
         xo = torch.empty((args.tokens, D_FF), dtype=torch.float32, device=dev)
         fn = lambda i: spark.ffn_predictor(q, k1s[i % len(k1s)], out=xo)
         unit = f"predictor GEMM, T={args.tokens}"
+    elif args.case == "topk_causal":
+        rows, d, k = 8 * 4096, 4096, 256
+        x = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+        out = torch.empty_like(x)
+        fn = lambda i: spark.stat_topk_soft_threshold_causal(x, k, n_q=4096, out=out)
+        unit = f"causal rows {rows} x {d}"
+    elif args.case == "huber_bwd":
+        rows, d, k = 8 * 4096, 4096, 256
+        x = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
+        g = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(6))
+        gx = torch.empty_like(x)
+        fn = lambda i: spark.stat_topk_huber_backward(x, g, k, 0.25, grad_x=gx)
+        unit = f"Huber backward rows {rows} x {d}"
     elif args.case == "topk":
         rows, d, k = 8 * 4096, 4096, 256
         x = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
@@ -651,6 +665,47 @@ def extra_workloads(spark, synthetic, torch, dev, base, copies, world, args, hbm
                                    "frac_of_hbm_peak": gbs / hbm_gbs,
                                    "traffic": profile_traffic("stat_topk_32768x4096.txt", TOPK_SOURCES),
                                    "note": "512 MiB read + 512 MiB written per call (> L2)"}
+    # the same rows under a causal mask (square scores of one 4096-token prompt per head): row i of a head
+    # sees i + 1 keys, rows with at most k of them pass through
+    tc = torch.empty(rows, dtype=torch.float32, device=dev)
+
+    def tkc():
+        rc = L.stat_topk_soft_threshold_causal(xs.data_ptr(), rows, d, k, 4096, 0, xo.data_ptr(), tc.data_ptr(),
+                                               _binding.stream_handle())
+        if rc != 0:
+            raise _binding.SparkError("stat_topk_soft_threshold_causal", rc)
+
+    ms, n = time_graph([tkc] * 2, 20, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    cbytes = 8 * (4096 * 4097 // 2) * 4 + rows * d * 4 + rows * 4  # visible entries read, all written, theta
+    gbs = cbytes / (ms * 1e-3) / 1e9
+    res["stat_topk_causal_32768x4096"] = {"rows_per_s": whole_job_rate(rows, ms, world), "ms_per_call": ms,
+                                          "achieved_GBs": gbs, "frac_of_hbm_peak": gbs / hbm_gbs,
+                                          "algorithmic_bytes": cbytes,
+                                          "traffic": profile_traffic("stat_topk_causal_32768x4096.txt", TOPK_SOURCES),
+                                          "note": "8 heads x 4096 queries x 4096 keys, causal: the visible "
+                                                  "entries (268 MB) read, every entry (537 MB) written"}
+    # backward of the Huber-smoothed operator on the same rows (delta = 0.25): x and the upstream
+    # gradient read, the gradient written, 12 bytes per element
+    gs = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(6))
+
+    def hb():
+        rc = L.stat_topk_huber_backward(xs.data_ptr(), gs.data_ptr(), rows, d, k, 0.25, xo.data_ptr(),
+                                        _binding.stream_handle())
+        if rc != 0:
+            raise _binding.SparkError("stat_topk_huber_backward", rc)
+
+    ms, n = time_graph([hb] * 2, 20, args.warmup, world)
+    ms = max_over_ranks(ms, world)
+    hbytes = rows * d * 12
+    gbs = hbytes / (ms * 1e-3) / 1e9
+    res["stat_topk_huber_backward_32768x4096"] = {
+        "rows_per_s": whole_job_rate(rows, ms, world), "ms_per_call": ms, "achieved_GBs": gbs,
+        "frac_of_hbm_peak": gbs / hbm_gbs, "algorithmic_bytes": hbytes,
+        "traffic": profile_traffic("stat_topk_huber_backward_32768x4096.txt", TOPK_SOURCES),
+        "note": "gradient of the Huber-smoothed statistical top-k (delta 0.25): x and grad_out read, grad_x "
+                "written (1.61 GB per call)"}
+    del gs
     return res
 
 

@@ -180,6 +180,48 @@ SPARK_API int stat_topk_soft_threshold(const float* x, int rows, int d, int k, f
                                        spark_stream_t stream);
 
 /*
+ * Huber-smoothed statistical top-k ("Statistical Top-k", Theorem 3.2: with a
+ * Huber smoothing the operator is continuously differentiable, for training).
+ * Reading of the smoothing: the ramp max{z, 0} of Soft-Threshold becomes
+ *   rho(z) = 0 (z <= 0),  z^2 / (2 delta) (0 < z < delta),  z - delta/2 (z >= delta)
+ * with z = x - theta(x), theta = mean + std * Q(1 - k/d) per row (population
+ * std); delta = 0 is the plain operator (stat_topk_soft_threshold).
+ *   stat_topk_huber:          out = rho(x - theta(x)), fp32 [rows][d]; out may equal x.
+ *   stat_topk_huber_backward: the gradient for an upstream gradient grad_out
+ *     (fp32 [rows][d]) of that output:
+ *       grad_x_j = w_j - W (1/d + Q (x_j - mean) / (d std)),
+ *       w = grad_out * rho'(x - theta),  W = sum_j w_j
+ *     (theta itself depends on every x_j through the row's mean and std; a
+ *     row with zero spread gets zero gradient).  grad_x may equal x or
+ *     grad_out (in place); other overlaps are SPARK_EINVAL.
+ * Require 0 < k < d, d >= 2, finite delta >= 0 and 4-byte aligned pointers.
+ * rows == 0 is a no-op.
+ */
+SPARK_API int stat_topk_huber(const float* x, int rows, int d, int k, float delta, float* out, spark_stream_t stream);
+SPARK_API int stat_topk_huber_backward(const float* x, const float* grad_out, int rows, int d, int k, float delta,
+                                       float* grad_x, spark_stream_t stream);
+
+/*
+ * Statistical top-k with soft threshold on causally masked score rows ("Spark
+ * Attention": each token attends to at most k tokens, so a query at position
+ * p works on min{k, p + 1} keys).  Row r of x (fp32 [rows][d]) is query
+ * r % n_q of its head, at position pos = offset + r % n_q, and sees its first
+ * n = min(d, pos + 1) entries:
+ *   k <  n: theta = mean + std * Q(1 - k/n) over those n entries (population
+ *           std), out = max(x - theta, 0) on them;
+ *   k >= n: every visible entry is kept: out = x on them, theta = -inf.
+ * Masked entries (index >= n) are written as 0 and do not influence the
+ * result (a row's last visible 16-byte group may be read whole).  theta_out
+ * (fp32 [rows], may be NULL) receives theta.  For the square causal scores of
+ * one prompt, n_q = d and offset = 0; for the last n_q queries of a longer
+ * context, offset = d - n_q.  out may equal x (in place); other overlaps are
+ * SPARK_EINVAL.  Requires k >= 1, n_q >= 1, offset >= 0, d >= 1, 4-byte
+ * aligned pointers.  rows == 0 is a no-op.
+ */
+SPARK_API int stat_topk_soft_threshold_causal(const float* x, int rows, int d, int k, int n_q, int offset,
+                                              float* out, float* theta_out, spark_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status of the
  * workspace used on that stream: SPARK_OK, SPARK_ETIMEOUT, or SPARK_ECUDA if
  * the stream reported a CUDA error.

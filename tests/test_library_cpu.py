@@ -88,3 +88,22 @@ def test_argument_checks_before_any_device_work(L):
     assert p(fake, fake, 2, 64, 36, 256, vp(1 << 30), null) == EALIGN  # r % 8
     assert p(fake, fake, 2, 64, 32, 256, vp((1 << 30) + 4), null) == EALIGN  # x_out alignment
     assert p(fake, fake, 2, 64, 32, 256, vp((1 << 20) + 64), null) == EINVAL  # x_out overlapping q
+    c = L.stat_topk_soft_threshold_causal
+    assert c(fake, 0, 64, 8, 64, 0, fake, null, null) == 0  # no rows: no-op
+    assert c(fake, 4, 64, 0, 64, 0, vp(1 << 30), null, null) == EINVAL  # k == 0
+    assert c(fake, 4, 64, 8, 0, 0, vp(1 << 30), null, null) == EINVAL  # n_q == 0
+    assert c(fake, 4, 64, 8, 64, -1, vp(1 << 30), null, null) == EINVAL  # offset < 0
+    assert c(null, 4, 64, 8, 64, 0, vp(1 << 30), null, null) == EINVAL
+    assert c(fake, 4, 64, 8, 64, 0, vp((1 << 20) + 16), null, null) == EINVAL  # partial overlap
+    assert c(fake, 4, 64, 8, 64, 0, vp(1 << 30), vp((1 << 20) + 8), null) == EINVAL  # theta inside x
+    assert c(vp((1 << 20) + 2), 4, 64, 8, 64, 0, vp(1 << 30), null, null) == EALIGN
+    h = L.stat_topk_huber
+    hb = L.stat_topk_huber_backward
+    assert h(fake, 0, 64, 8, 0.1, fake, null) == 0  # no rows: no-op
+    assert h(fake, 4, 64, 0, 0.1, vp(1 << 30), null) == EINVAL  # k == 0
+    assert h(fake, 4, 64, 8, -0.1, vp(1 << 30), null) == EINVAL  # negative delta
+    assert h(fake, 4, 64, 8, float("inf"), vp(1 << 30), null) == EINVAL
+    assert h(fake, 4, 64, 8, 0.1, vp((1 << 20) + 16), null) == EINVAL  # partial overlap
+    assert hb(fake, vp(1 << 24), 4, 64, 64, 0.1, vp(1 << 30), null) == EINVAL  # k == d
+    assert hb(fake, vp(1 << 24), 4, 64, 8, 0.1, vp((1 << 24) + 16), null) == EINVAL  # grad_x inside grad_out
+    assert hb(vp((1 << 20) + 2), vp(1 << 24), 4, 64, 8, 0.1, vp(1 << 30), null) == EALIGN
