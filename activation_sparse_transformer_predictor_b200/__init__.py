@@ -20,7 +20,7 @@ from ._binding import SparkError
 
 __all__ = ["ffn_forward", "ffn_forward_debug", "ffn_predictor", "ffn_decode_stack", "stat_topk_soft_threshold",
            "stat_topk_soft_threshold_causal", "stat_topk_huber", "stat_topk_huber_backward", "query_status", "release_workspace",
-           "topk_quantile", "set_wait_limit_ns", "selftest_wait_timeout", "SparkError"]
+           "topk_quantile", "set_wait_limit_ns", "selftest_wait_timeout", "debug_violations", "SparkError"]
 
 
 def _require(t, name, dtype, ndim=None):
@@ -208,6 +208,16 @@ def stat_topk_huber_backward(x, grad_out, k: int, delta: float, grad_x=None, str
 def query_status(stream=None) -> int:
     """Synchronise the stream and return (and clear) the device status code."""
     return int(_binding.lib().spark_query_status(_binding.stream_handle(stream)))
+
+
+def debug_violations() -> int:
+    """Failed bounds checks since the previous call in the current library
+    (cleared by the call); -1 in the release build.  Use inside
+    ``_binding.using_library(_binding.debug_lib())`` to read the checked build."""
+    n = int(_binding.lib().spark_debug_violations())
+    if n < -1:
+        raise SparkError("spark_debug_violations", n)
+    return n
 
 
 def release_workspace() -> None:

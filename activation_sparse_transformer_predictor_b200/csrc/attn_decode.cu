@@ -37,6 +37,12 @@
 #include "spark_internal.h"
 
 namespace spark {
+
+#ifdef SPARK_DEBUG
+// bounds-check violations of this file's kernels (see SPARK_CHECK)
+static __device__ unsigned g_bounds_violations;
+#endif
+
 namespace {
 
 constexpr int kAThreads = 256;
@@ -248,7 +254,8 @@ __global__ void __launch_bounds__(kAThreads, 2) attn_decode_kernel(const AttnPar
     const int i = b + lane;
     const bool act = i < nk && ss[i] > theta;
     const unsigned ball = __ballot_sync(0xffffffffu, act);
-    if (act) list[cnt + __popc(ball & ((1u << lane) - 1u))] = i;
+    const int slot = cnt + __popc(ball & ((1u << lane) - 1u));
+    if (act && SPARK_CHECK(slot < L.seg)) list[slot] = i;
     cnt += __popc(ball);
   }
   __syncwarp();
@@ -264,6 +271,7 @@ __global__ void __launch_bounds__(kAThreads, 2) attn_decode_kernel(const AttnPar
 #pragma unroll
     for (int u = 0; u < kGather; ++u) {
       idx[u] = jb + u < cnt ? list[jb + u] : -1;
+      if (idx[u] >= 0 && !SPARK_CHECK(idx[u] < nk && j0 + idx[u] < p.n_ctx)) idx[u] = -1;
       const size_t row = static_cast<size_t>(j0 + max(idx[u], 0)) * D;
       kv[u] = (idx[u] >= 0 && lane < cpk2) ? ldg_ro(Kg + row + p.r + lane * 8) : make_uint4(0, 0, 0, 0);
       vv[u] = (idx[u] >= 0 && lane < cpr) ? ldg_ro(Vg + row + lane * 8) : make_uint4(0, 0, 0, 0);
@@ -376,6 +384,23 @@ cudaError_t launch_attn_decode(const AttnArgs& a, int num_sms, cudaStream_t stre
   cfg.numAttrs = 1;
   (void)num_sms;
   return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
+
+// ---------------------------------------------------------------- debug builds
+unsigned take_bounds_violations_attention(bool clear) {
+#ifdef SPARK_DEBUG
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bounds_violations, sizeof v) != cudaSuccess ||
+      (clear && cudaMemcpyToSymbol(g_bounds_violations, &zero, sizeof zero) != cudaSuccess)) {
+    cudaGetLastError();
+    return 0xffffffffu;
+  }
+  return v;
+#else
+  (void)clear;
+  return 0;
+#endif
 }
 
 }  // namespace spark

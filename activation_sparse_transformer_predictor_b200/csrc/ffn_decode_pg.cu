@@ -35,6 +35,12 @@
 #include "spark_internal.h"
 
 namespace spark {
+
+#ifdef SPARK_DEBUG
+// bounds-check violations of this file's kernels (see SPARK_CHECK)
+static __device__ unsigned g_bounds_violations;
+#endif
+
 namespace {
 
 constexpr int kPWarps = 8;
@@ -368,7 +374,7 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
       const bool act = i < nr && x > th;
       const unsigned ball = __ballot_sync(0xffffffffu, act);
       const int slot = cnt + __popc(ball & ((1u << lane) - 1u));
-      if (act) {
+      if (act && SPARK_CHECK(slot < nr)) {
         act_i[slot] = n0 + i;
         act_h[slot] = x;  // x for now; h = GELU(x - theta) a below
       }
@@ -402,7 +408,7 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
 #pragma unroll
       for (int cp = 0; cp < CPT; ++cp) {
         const int ch = tid + cp * kGThreads;
-        v[cp][u] = (j0 + u < nact && ch < nco)
+        v[cp][u] = (j0 + u < nact && ch < nco && SPARK_CHECK(act_i[j0 + u] < p.d_ff))
                        ? ldg_ro128(p.V + static_cast<size_t>(act_i[j0 + u]) * D + ch * 8)
                        : make_uint4(0, 0, 0, 0);
       }
@@ -413,6 +419,7 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
       for (int j = warp; j < nact; j += 2 * kGWarps) {
         const int jb = j + kGWarps;
         const bool hasb = jb < nact;
+        if (!SPARK_CHECK(act_i[j] < p.d_ff && act_i[hasb ? jb : j] < p.d_ff)) continue;
         const uint16_t* ra = p.K2 + static_cast<size_t>(act_i[j]) * p.d2;
         const uint16_t* rb = p.K2 + static_cast<size_t>(act_i[hasb ? jb : j]) * p.d2;
         uint4 ka[KCH], kb[KCH];
@@ -462,6 +469,7 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
       }
     }
   }
+  if (!SPARK_CHECK(c < p.n_slices && p.n_slices <= kMaxSlices)) return;
   float* mypart = p.part + static_cast<size_t>(c) * D;
 #pragma unroll
   for (int cp = 0; cp < CPT; ++cp) {
@@ -656,6 +664,23 @@ cudaError_t launch_decode_pg(const DecodePgPlan& pl, const DecodePgArgs& a, cuda
   cfg.blockDim = dim3(kRThreads);
   cfg.dynamicSmemBytes = 0;
   return cudaLaunchKernelEx(&cfg, decode_reduce_kernel, p);
+}
+
+
+// ---------------------------------------------------------------- debug builds
+unsigned take_bounds_violations_decode(bool clear) {
+#ifdef SPARK_DEBUG
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bounds_violations, sizeof v) != cudaSuccess ||
+      (clear && cudaMemcpyToSymbol(g_bounds_violations, &zero, sizeof zero) != cudaSuccess)) {
+    cudaGetLastError();
+    return 0xffffffffu;
+  }
+  return v;
+#else
+  (void)clear;
+  return 0;
+#endif
 }
 
 }  // namespace spark

@@ -34,6 +34,12 @@
 
 namespace spark {
 
+#ifdef SPARK_DEBUG
+// bounds-check violations of this file's kernels (see SPARK_CHECK)
+static __device__ unsigned g_bounds_violations;
+#endif
+
+
 namespace {
 
 constexpr int kWarps = 8;
@@ -354,8 +360,8 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_fused_kernel(const KPar
       wcnt[kWarps] = run;
     }
     __syncthreads();
-    if (any) {
-      const int pos = wcnt[warp] + __popc(ballot & ((1u << lane) - 1u));
+    const int pos = wcnt[warp] + __popc(ballot & ((1u << lane) - 1u));
+    if (any && SPARK_CHECK(pos < nr)) {
       uidx[pos] = li;
 #pragma unroll
       for (int t = 0; t < kFusedMaxTokens; ++t)
@@ -387,7 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1) spark_ffn_fused_kernel(const KPar
       }
       __syncwarp();
       for (int u = lane; u < nb; u += 32) {
-        const size_t row = static_cast<size_t>(n0 + uidx[b0 + u]);
+        // (a failed check copies the slice's first row so the byte count still
+        // matches the barrier's expected transaction bytes)
+        const int li = uidx[b0 + u];
+        const size_t row = static_cast<size_t>(n0 + (SPARK_CHECK(li >= 0 && n0 + li < p.d_ff) ? li : 0));
         unsigned char* dst = region_a + static_cast<size_t>(u) * row_bytes;
         bulk_g2s(dst, p.K2 + row * p.d2, p.d2 * 2, &bars[pbar]);
         bulk_g2s(dst + static_cast<size_t>(p.d2) * 2, p.V + row * p.d_model, p.d_model * 2, &bars[pbar]);
@@ -648,6 +657,23 @@ cudaError_t launch_fused(const FusedPlan& pl, const FusedArgs& a, cudaStream_t s
   cfg.numAttrs = 1;
   if (a.T == 1) return cudaLaunchKernelEx(&cfg, spark_ffn_fused_kernel<1>, p);
   return cudaLaunchKernelEx(&cfg, spark_ffn_fused_kernel<2>, p);
+}
+
+
+// ---------------------------------------------------------------- debug builds
+unsigned take_bounds_violations_fused(bool clear) {
+#ifdef SPARK_DEBUG
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bounds_violations, sizeof v) != cudaSuccess ||
+      (clear && cudaMemcpyToSymbol(g_bounds_violations, &zero, sizeof zero) != cudaSuccess)) {
+    cudaGetLastError();
+    return 0xffffffffu;
+  }
+  return v;
+#else
+  (void)clear;
+  return 0;
+#endif
 }
 
 }  // namespace spark

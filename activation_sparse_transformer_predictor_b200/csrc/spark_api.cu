@@ -515,6 +515,25 @@ SPARK_API int stat_topk_soft_threshold_causal(const float* x, int rows, int d, i
   return SPARK_OK;
 }
 
+// Failed index checks counted by the kernels of the current device (bounds-check
+// build; 0 in release builds), cleared with `clear`; -1 if reading them failed.
+static long long bounds_violations(bool clear) {
+  const unsigned counts[4] = {take_bounds_violations_decode(clear), take_bounds_violations_fused(clear),
+                              take_bounds_violations_prefill(clear), take_bounds_violations_attention(clear)};
+  long long total = 0;
+  for (unsigned c : counts) {
+    if (c == 0xffffffffu) return -1;
+    total += c;
+  }
+  return total;
+}
+
+static int with_bounds_status(int status) {
+  if (status != SPARK_OK) return status;
+  const long long v = bounds_violations(false);
+  return v < 0 ? SPARK_ECUDA : v > 0 ? SPARK_EBOUNDS : SPARK_OK;
+}
+
 SPARK_API int spark_query_status(spark_stream_t stream_) {
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (cudaStreamSynchronize(stream) != cudaSuccess) {
@@ -529,12 +548,13 @@ SPARK_API int spark_query_status(spark_stream_t stream_) {
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     auto it = g_workspaces.find({dev, stream});
-    if (it == g_workspaces.end() || it->second.ptr == nullptr) return na;
-    ptr = it->second.ptr;
+    if (it == g_workspaces.end() || it->second.ptr == nullptr) ptr = nullptr;
+    else ptr = it->second.ptr;
   }
+  if (ptr == nullptr) return with_bounds_status(na);
   DeviceControl ctl;
   if (cudaMemcpy(&ctl, ptr, sizeof ctl, cudaMemcpyDeviceToHost) != cudaSuccess) return SPARK_ECUDA;
-  if (ctl.status == kDevOk && ctl.abort == 0) return na;
+  if (ctl.status == kDevOk && ctl.abort == 0) return with_bounds_status(na);
   if (cudaMemset(ptr, 0, sizeof ctl) != cudaSuccess) return SPARK_ECUDA;  // barrier state too
   return ctl.status == kDevTimeout ? SPARK_ETIMEOUT : SPARK_ECUDA;
 }
@@ -564,6 +584,7 @@ SPARK_API const char* spark_status_string(int status) {
     case SPARK_ETIMEOUT: return "SPARK_ETIMEOUT: device wait timed out";
     case SPARK_EDEVICE: return "SPARK_EDEVICE: device is not sm_100";
     case SPARK_ESCRATCH: return "SPARK_ESCRATCH: problem exceeds the fixed no-allocation scratch";
+    case SPARK_EBOUNDS: return "SPARK_EBOUNDS: a kernel index check failed (bounds-check build)";
     default: return "SPARK_UNKNOWN";
   }
 }
@@ -609,6 +630,20 @@ SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream) {
   g_wait_limit_ns = saved;
   cudaFreeAsync(buf, s);
   return rc;
+}
+
+SPARK_API int spark_debug_violations(void) {
+#ifdef SPARK_DEBUG
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  const long long total = bounds_violations(true);
+  if (total < 0) return SPARK_ECUDA;
+  return total > 0x7fffffffll ? 0x7fffffff : static_cast<int>(total);
+#else
+  return -1;
+#endif
 }
 
 SPARK_API int spark_version(void) { return 100; }

@@ -15,7 +15,7 @@ namespace spark {
 // spark_query_status.  The arrival counters are reset by the last CTA to leave
 // each launch, so every launch starts from zeros.
 // ----------------------------------------------------------------------------
-enum DeviceError : unsigned { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };
+enum DeviceError : unsigned { kDevOk = 0, kDevTimeout = 1 };
 
 struct DeviceControl {
   unsigned int status;      // first device error recorded (0 = none)
@@ -108,6 +108,25 @@ __device__ __forceinline__ bool wait_count_geq(DeviceControl* ctl, const unsigne
     }
   }
 }
+
+// ----------------------------------------------------------------------------
+// Debug builds (compiled with SPARK_DEBUG: libspark_debug.so) check indices the
+// kernels compute -- gathered neuron and key rows, active counts, partial-output
+// slots, operand block numbers -- before using them.  A failed check counts into
+// the word g_bounds_violations that every .cu file using SPARK_CHECK defines
+// (static __device__), and the guarded access is skipped; nothing traps.
+// spark_debug_violations() reads and clears the words.  Release builds compile
+// SPARK_CHECK(c) to `true` without evaluating c.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ bool bounds_check(bool ok, unsigned* counter) {
+  if (!ok) atomicAdd(counter, 1u);
+  return ok;
+}
+#ifdef SPARK_DEBUG
+#define SPARK_CHECK(cond) ::spark::bounds_check(static_cast<bool>(cond), &g_bounds_violations)
+#else
+#define SPARK_CHECK(cond) true
+#endif
 
 // ----------------------------------------------------------------------------
 // mbarrier + bulk copy (TMA engine, 1-D form) wrappers.

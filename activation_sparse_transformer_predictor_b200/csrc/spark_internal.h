@@ -19,6 +19,15 @@ unsigned long long wait_limit_ns();
 // was never set up on `dev`.
 int noalloc_take_status(int dev);
 
+// ---------------------------------------------------------------- debug builds
+// Failed index checks counted by each file's kernels (bounds-check build) since
+// the last clearing read; 0xffffffff if the read failed; 0 without a CUDA call
+// in release builds.
+unsigned take_bounds_violations_decode(bool clear);
+unsigned take_bounds_violations_fused(bool clear);
+unsigned take_bounds_violations_prefill(bool clear);
+unsigned take_bounds_violations_attention(bool clear);
+
 // ---------------------------------------------------------------- stat top-k
 cudaError_t launch_stat_topk(const float* x, float* out, int rows, int d, float Q, cudaStream_t stream);
 cudaError_t launch_stat_topk_huber(const float* x, float* out, int rows, int d, float Q, float delta,

@@ -17,7 +17,10 @@
 //
 // With independent tokens the union of the per-token active sets covers almost
 // every neuron once a 128-token tile is formed (1 - 0.92^128), so the masked
-// products run as dense tiles.  h is split in two bf16 parts because a single
+// products run as dense tiles.  Restricting GEMM 3 to the union's V rows -- by
+// gathering them (TMA tile::gather4 over compacted positions) or by zeroing the
+// other rows in shared memory before the product -- measured slower at every
+// prompt length, so every row of K2 and V is read (and must be finite).  h is split in two bf16 parts because a single
 // bf16 rounding of h would add ~1.7e-3 relative error on top of the bf16 output
 // rounding and break the 2e-3 relative-L2 target.
 //
@@ -36,6 +39,12 @@
 #include "spark_internal.h"
 
 namespace spark {
+
+#ifdef SPARK_DEBUG
+// bounds-check violations of this file's kernels (see SPARK_CHECK)
+static __device__ unsigned g_bounds_violations;
+#endif
+
 namespace {
 
 constexpr int BM = 128;
@@ -201,7 +210,8 @@ __device__ __forceinline__ uint4* h_block(uint16_t* h, const GemmParams& p, int 
 // GEMM 2 epilogue: float4 group i of row `row` of the scores [nb, nb + 128), as
 // GEMM 1 stored them (N is a multiple of 16: a group of four is wholly inside)
 __device__ __forceinline__ float4 gate_x(const GemmParams& p, const float4* tile, int row, int nb, int i) {
-  return nb + 4 * i < p.N ? __ldcg(tile + i * BM + row) : make_float4(0.f, 0.f, 0.f, 0.f);
+  return nb + 4 * i < p.N && SPARK_CHECK(nb / BN < p.xt_tiles_n) ? __ldcg(tile + i * BM + row)
+                                                                  : make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
@@ -332,9 +342,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         mbar_arrive_expect_tx(&full[stage], kStageBytes);
         unsigned char* sb = sa + kAB * (DUAL ? 2 : 1);
         if (EPI == kEpiOut) {
-          // h_hi and h_lo blocks: already in the operand layout
-          bulk_g2s(sa, h_block(p.h_hi, p, tm, kb), kHBlockBytes, &full[stage]);
-          bulk_g2s(sa + kABytes, h_block(p.h_lo, p, tm, kb), kHBlockBytes, &full[stage]);
+          // h_hi and h_lo blocks: already in the operand layout (a failed check
+          // copies block (0, 0) so the byte count still matches the barrier)
+          const bool hb_ok = SPARK_CHECK(tm < p.tiles_m && kb < p.h_kb);
+          bulk_g2s(sa, h_block(p.h_hi, p, hb_ok ? tm : 0, hb_ok ? kb : 0), kHBlockBytes, &full[stage]);
+          bulk_g2s(sa + kABytes, h_block(p.h_lo, p, hb_ok ? tm : 0, hb_ok ? kb : 0), kHBlockBytes, &full[stage]);
         } else {
           tma_load_2d(sa, &tmA, kb * BK, tm * BM, &full[stage]);
           if (DUAL) tma_load_2d(sa + kABytes, &tmA2, kb * BK, tm * BM, &full[stage]);
@@ -489,7 +501,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                 sum += v[j];
                 ++cnt;
               }
-            if (row_ok && n < p.N && p.Xt != nullptr) {
+            if (row_ok && n < p.N && p.Xt != nullptr && SPARK_CHECK(tm < p.tiles_m && nb / BN < p.xt_tiles_n)) {
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4)
                 xt[(c / 4 + q4) * BM + row] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
@@ -534,10 +546,12 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                                  xr[c / 4 + 1].x, xr[c / 4 + 1].y, xr[c / 4 + 1].z, xr[c / 4 + 1].w,
                                  xr[c / 4 + 2].x, xr[c / 4 + 2].y, xr[c / 4 + 2].z, xr[c / 4 + 2].w,
                                  xr[c / 4 + 3].x, xr[c / 4 + 3].y, xr[c / 4 + 3].z, xr[c / 4 + 3].w};
-            // every row of the block is stored (rows >= M only ever reach output
-            // rows >= M); neurons in [N, next multiple of 64) are stored as zeros,
-            // since GEMM 3 multiplies them with the zero rows TMA fills in for V
-            if (n >= (p.N + BK - 1) / BK * BK) continue;
+            // rows < M are stored (rows >= M only ever reach output rows >= M,
+            // whatever the block holds there); neurons in [N, next multiple of 64)
+            // are stored as zeros, since GEMM 3 multiplies them with the zero rows
+            // TMA fills in for V
+            if (n >= (p.N + BK - 1) / BK * BK || !row_ok) continue;
+            if (!SPARK_CHECK(tm < p.tiles_m && n / BK < p.h_kb)) continue;
             const bool col_ok = n < p.N;
             uint32_t hi[8], lo[8];
 #pragma unroll
@@ -591,6 +605,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                 if (n + j < p.N) orow[n + j] = f2bf(v[j]);
             }
           } else {
+            if (!SPARK_CHECK(split < p.split_k)) continue;
             float* prow = p.part + (static_cast<size_t>(split) * p.M + m) * p.N;
             if (n + 16 <= p.N) {
               float4* d = reinterpret_cast<float4*>(prow + n);
@@ -929,6 +944,23 @@ cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, 
   }
   if (a64) return launch_gemm<kEpiPredictor, false, false, 8, false, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
   return launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+}
+
+
+// ---------------------------------------------------------------- debug builds
+unsigned take_bounds_violations_prefill(bool clear) {
+#ifdef SPARK_DEBUG
+  unsigned v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_bounds_violations, sizeof v) != cudaSuccess ||
+      (clear && cudaMemcpyToSymbol(g_bounds_violations, &zero, sizeof zero) != cudaSuccess)) {
+    cudaGetLastError();
+    return 0xffffffffu;
+  }
+  return v;
+#else
+  (void)clear;
+  return 0;
+#endif
 }
 
 }  // namespace spark

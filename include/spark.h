@@ -60,7 +60,8 @@ typedef enum {
   SPARK_ENOMEM = -4,   /* workspace could not be allocated (or growth requested during capture) */
   SPARK_ETIMEOUT = -5, /* a device-side bounded wait ran out (reported by spark_query_status) */
   SPARK_EDEVICE = -6,  /* current device is not compute capability 10.x (B200 / sm_100a) */
-  SPARK_ESCRATCH = -7  /* spark_ffn_forward_noalloc: problem needs more than its fixed scratch */
+  SPARK_ESCRATCH = -7, /* spark_ffn_forward_noalloc: problem needs more than its fixed scratch */
+  SPARK_EBOUNDS = -8   /* bounds-check build only: a kernel index check failed (spark_query_status) */
 } spark_status;
 
 /*
@@ -83,6 +84,16 @@ SPARK_API int spark_ffn_forward(const void* q, const void* K1, const void* K2, c
  * q and out are bf16 [n_tokens][d_model]; every token gets its own threshold and
  * active set.  n_tokens == 0 is a no-op returning SPARK_OK; n_tokens < 0 is
  * SPARK_EINVAL.
+ *
+ * Which weight rows are read: up to 4 tokens, all of K1 and only the rows of K2
+ * and V that some token's active set uses.  From 5 tokens on, the tensor-core
+ * path reads all of K1, K2 and V in dense tiles (the masked products multiply
+ * zero h entries): the union of independent tokens' active sets covers most
+ * neurons from a few tokens on (1 - (1 - k/d_ff)^T), and reading only the
+ * union's rows -- gathered, or zeroed in shared memory before the product --
+ * measured slower than the dense tiles on B200 at every prompt length.  So from
+ * 5 tokens on every row of K2 and V must be finite: a NaN or Inf in a row that no
+ * token uses still reaches out (0 * NaN is NaN).
  */
 SPARK_API int spark_ffn_forward_tokens(const void* q, const void* K1, const void* K2,
                                        const void* V, int n_tokens, int d_model, int r, int d_ff,
@@ -224,7 +235,10 @@ SPARK_API int stat_topk_soft_threshold_causal(const float* x, int rows, int d, i
 /*
  * Synchronises `stream`, then returns and clears the device status of the
  * workspace used on that stream: SPARK_OK, SPARK_ETIMEOUT, or SPARK_ECUDA if
- * the stream reported a CUDA error.
+ * the stream reported a CUDA error.  In the bounds-check build
+ * (libspark_debug.so) it returns SPARK_EBOUNDS when no other error is pending
+ * and a kernel of the current device has counted a failed index check since
+ * the last spark_debug_violations(), which reads and clears that count.
  */
 SPARK_API int spark_query_status(spark_stream_t stream);
 
@@ -313,6 +327,22 @@ SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream);
 SPARK_API int spark_ffn_forward_noalloc(const void* q, const void* K1, const void* K2, const void* V,
                                         int d_model, int r, int d_ff, int k, void* out,
                                         spark_stream_t stream);
+
+/*
+ * Bounds-check build.  libspark_debug.so is this library compiled with
+ * SPARK_DEBUG: its kernels check the indices they compute before using them
+ * (gathered neuron rows against d_ff, active counts against the slice,
+ * gathered key rows against n_ctx, partial-output slots, GEMM operand blocks)
+ * and skip an access whose check fails, counting it; they never trap.  The
+ * results of a run without violations are bit-identical to libspark.so's.
+ *
+ * Returns the number of failed checks since the previous call (summed over the
+ * kernels of the current device) and clears the count; synchronises the device
+ * first.  While the count is nonzero, spark_query_status reports SPARK_EBOUNDS.
+ * Returns -1 in the release library, whose kernels contain no checks, and
+ * SPARK_ECUDA (-3) if reading the counts failed.
+ */
+SPARK_API int spark_debug_violations(void);
 
 /* Library version: major*10000 + minor*100 + patch. */
 SPARK_API int spark_version(void);

@@ -70,8 +70,9 @@ def test_gemma_small_batches(T):
     run_parity(*GEMMA, T=T, layer=10 + T)
 
 
-@pytest.mark.parametrize("T", [64, 256])
+@pytest.mark.parametrize("T", [5, 64, 100, 128, 129, 256])
 def test_gemma_prefill(T):
+    """One 128-token band up to 128 tokens, two from 129 on; 64-row token boxes up to 64 tokens."""
     run_parity(*GEMMA, T=T, layer=20 + T)
 
 
@@ -125,11 +126,21 @@ def test_degenerate_rows_select_nothing():
     K1c = K1[:1].repeat(d_ff, 1).contiguous()  # identical predictor rows: constant x
     res = spark.ffn_forward_debug(dev["q"], K1c, dev["K2"], dev["V"], k)
     assert int(res["active"].sum()) == 0 and torch.all(res["out"] == 0)
+    # prefill with an empty union (every token's x constant): h is zero everywhere
+    d_model, r, d_ff, k = GEMMA
+    dev, _ = make_layer(d_model, r, d_ff, 12, layer=4)
+    K1c = dev["K1"][:1].repeat(d_ff, 1).contiguous()
+    res = spark.ffn_forward_debug(dev["q"], K1c, dev["K2"], dev["V"], k)
+    torch.cuda.synchronize()
+    assert spark.query_status() == 0
+    assert int(res["active"].sum()) == 0 and torch.all(res["out"] == 0)
 
 
-@pytest.mark.parametrize("shape,T", [(GEMMA, 1), (GEMMA, 4), (TINY, 4)])
+@pytest.mark.parametrize("shape,T", [(GEMMA, 1), (GEMMA, 4), (TINY, 4), (TINY, 3)])
 def test_poisoned_inactive_rows_are_never_read(shape, T):
-    """NaN in every K2 / V row outside the active set leaves out bit-identical."""
+    """NaN in every K2 / V row outside the union of the tokens' active sets leaves out bit-identical:
+    decode and small batches (T <= 4) read only the active rows.  (Prefill, T >= 5, reads every row by
+    design: see spark.h.)"""
     d_model, r, d_ff, k = shape
     dev, _ = make_layer(d_model, r, d_ff, T, layer=5)
     res = spark.ffn_forward_debug(dev["q"], dev["K1"], dev["K2"], dev["V"], k)

@@ -107,3 +107,13 @@ def test_argument_checks_before_any_device_work(L):
     assert hb(fake, vp(1 << 24), 4, 64, 64, 0.1, vp(1 << 30), null) == EINVAL  # k == d
     assert hb(fake, vp(1 << 24), 4, 64, 8, 0.1, vp((1 << 24) + 16), null) == EINVAL  # grad_x inside grad_out
     assert hb(vp((1 << 20) + 2), vp(1 << 24), 4, 64, 8, 0.1, vp(1 << 30), null) == EALIGN
+
+
+def test_debug_library_exports_the_same_symbols(L):
+    """libspark_debug.so (SPARK_DEBUG) declares the same C ABI; the release
+    library answers -1 to spark_debug_violations without touching a device."""
+    D = _binding.debug_lib()
+    for name in _declared_functions():
+        assert hasattr(D, name), name
+    assert D.spark_version() == L.spark_version()
+    assert L.spark_debug_violations() == -1
