@@ -123,6 +123,23 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// 32 consecutive fp32 columns of this thread's TMEM lane (one wait).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
 // 16 consecutive fp32 columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
   uint32_t r[16];
@@ -497,66 +514,76 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       if (EPI == kEpiPredictor) {
 #pragma unroll 1
         for (int h = 0; h < kBTiles; ++h) {
-          // one 128-column half: moments about its mean (two passes over TMEM)
+          // one 128-column half, 32 columns per TMEM load; its moments about its
+          // mean (a second pass over TMEM) unless moments are not wanted
           const int nb = n_base + h * BN;
           const uint32_t ta = taddr + static_cast<uint32_t>(h * BN);
           float4* xt = xt_tile(p, tm, nb);
           float sum = 0.f;
           int cnt = 0;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 16) {
-            tmem_ld16(ta + c, v);
-            const int n = nb + c;
+          for (int c = 0; c < BN; c += 32) {
+            float w[32];
+            tmem_ld32(ta + c, w);
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (n + j < p.N) {
-                sum += v[j];
-                ++cnt;
+            for (int s = 0; s < 32; s += 16) {
+              const float* v = w + s;
+              const int n = nb + c + s;
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                if (n + j < p.N) {
+                  sum += v[j];
+                  ++cnt;
+                }
+              if (row_ok && n < p.N && p.Xt != nullptr && SPARK_CHECK(tm < p.tiles_m && nb / BN < p.xt_tiles_n)) {
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4)
+                  xt[((c + s) / 4 + q4) * BM + row] =
+                      make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
               }
-            if (row_ok && n < p.N && p.Xt != nullptr && SPARK_CHECK(tm < p.tiles_m && nb / BN < p.xt_tiles_n)) {
+              if (p.X != nullptr) {
+                // through shared memory: lane l's 16 values go to row l of a 32 x 16
+                // staging block (16-byte chunks xor-swizzled), read back so that one
+                // store instruction covers 8 rows x 64 contiguous bytes
+                float4* stg = reinterpret_cast<float4*>(smem + STAGES * kStageBytes + 256) + quarter * 128;
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4)
-                xt[(c / 4 + q4) * BM + row] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-            }
-            if (p.X != nullptr) {
-              // through shared memory: lane l's 16 values go to row l of a 32 x 16
-              // staging block (16-byte chunks xor-swizzled), read back so that one
-              // store instruction covers 8 rows x 64 contiguous bytes
-              float4* stg = reinterpret_cast<float4*>(smem + STAGES * kStageBytes + 256) + quarter * 128;
+                for (int q4 = 0; q4 < 4; ++q4)
+                  stg[lane * 4 + (q4 ^ ((lane >> 1) & 3))] =
+                      make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+                __syncwarp();
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4)
-                stg[lane * 4 + (q4 ^ ((lane >> 1) & 3))] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-              __syncwarp();
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const int rr = i * 8 + (lane >> 2), q4 = lane & 3;
-                const float4 val = stg[rr * 4 + (q4 ^ ((rr >> 1) & 3))];
-                const int mr = tm * BM + quarter * 32 + rr;
-                const int nc = n + 4 * q4;
-                if (mr < p.M) {
-                  float* dst = p.X + static_cast<size_t>(mr) * p.N + nc;
-                  if (nc + 4 <= p.N) {
-                    *reinterpret_cast<float4*>(dst) = val;
-                  } else {
-                    if (nc < p.N) dst[0] = val.x;
-                    if (nc + 1 < p.N) dst[1] = val.y;
-                    if (nc + 2 < p.N) dst[2] = val.z;
+                for (int i = 0; i < 4; ++i) {
+                  const int rr = i * 8 + (lane >> 2), q4 = lane & 3;
+                  const float4 val = stg[rr * 4 + (q4 ^ ((rr >> 1) & 3))];
+                  const int mr = tm * BM + quarter * 32 + rr;
+                  const int nc = n + 4 * q4;
+                  if (mr < p.M) {
+                    float* dst = p.X + static_cast<size_t>(mr) * p.N + nc;
+                    if (nc + 4 <= p.N) {
+                      *reinterpret_cast<float4*>(dst) = val;
+                    } else {
+                      if (nc < p.N) dst[0] = val.x;
+                      if (nc + 1 < p.N) dst[1] = val.y;
+                      if (nc + 2 < p.N) dst[2] = val.z;
+                    }
                   }
                 }
+                __syncwarp();
               }
-              __syncwarp();
             }
           }
+          if (p.moments == nullptr) continue;
           const float mean = cnt > 0 ? sum / static_cast<float>(cnt) : 0.f;
           float m2 = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 16) {
-            tmem_ld16(ta + c, v);
+          for (int c = 0; c < BN; c += 32) {
+            float w[32];
+            tmem_ld32(ta + c, w);
             const int n = nb + c;
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
+            for (int j = 0; j < 32; ++j)
               if (n + j < p.N) {
-                const float d = v[j] - mean;
+                const float d = w[j] - mean;
                 m2 += d * d;
               }
           }
@@ -786,10 +813,7 @@ size_t align256(size_t v) { return (v + 255) / 256 * 256; }
 
 }  // namespace
 
-size_t predictor_workspace_bytes(int T, int d_ff) {
-  const int tiles_n = (d_ff + BN - 1) / BN;
-  return align256(sizeof(DeviceControl)) + align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));
-}
+size_t predictor_workspace_bytes(int, int) { return align256(sizeof(DeviceControl)); }
 
 size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms) {
   const int tiles_n = (d_ff + BN - 1) / BN;
@@ -946,8 +970,9 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
 
 // GEMM 1 alone (the low-rank predictor x = K1^T q[:r] for T tokens), the same
 // kernel and unit choice as in launch_prefill, writing x row-major to x_out
-// instead of the tiled copy GEMM 2 reads; the per-tile moments go to the
-// workspace as usual.
+// instead of the tiled copy GEMM 2 reads, and no tile moments (measured
+// 12.8 -> 11.9 us at T = 256 together with 32-column TMEM loads).  The
+// workspace holds only the control block.
 cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, int r, int d_ff, float* x_out,
                              void* workspace, unsigned long long wait_limit_ns, int num_sms, cudaStream_t stream) {
   const int tiles_n = (d_ff + BN - 1) / BN;
@@ -963,7 +988,7 @@ cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, 
   g.X = x_out;
   g.Xt = nullptr;
   g.xt_tiles_n = tiles_n;
-  g.moments = reinterpret_cast<float2*>(ws + align256(sizeof(DeviceControl)));
+  g.moments = nullptr;  // x only
   g.mom_stride = tiles_n;
   g.M = T;
   g.N = d_ff;
