@@ -18,7 +18,7 @@ from __future__ import annotations
 from . import _binding
 from ._binding import SparkError
 
-__all__ = ["ffn_forward", "ffn_forward_debug", "ffn_predictor", "ffn_decode_stack", "stat_topk_soft_threshold",
+__all__ = ["ffn_forward", "ffn_forward_host", "ffn_forward_debug", "ffn_predictor", "ffn_decode_stack", "stat_topk_soft_threshold",
            "stat_topk_soft_threshold_causal", "stat_topk_huber", "stat_topk_huber_backward", "query_status", "release_workspace",
            "topk_quantile", "set_wait_limit_ns", "selftest_wait_timeout", "debug_violations", "SparkError"]
 
@@ -67,6 +67,29 @@ def ffn_forward(q, K1, K2, V, k: int, out=None, stream=None):
                                         d_ff, int(k), out.data_ptr(), st)
         _binding.check("spark_ffn_forward_tokens", rc)
     return out
+
+
+def ffn_forward_host(q_host, K1, K2, V, k: int, out_host=None, stream=None):
+    """spark_ffn_forward_host: q_host and out_host are bf16 CPU tensors ([d_model] or [T, d_model]),
+    pinned for an asynchronous call; the weights are CUDA tensors.  The output copy is enqueued on the
+    stream: synchronise before reading out_host.  Returns out_host."""
+    import torch
+    if q_host.device.type != "cpu" or q_host.dtype != torch.bfloat16 or not q_host.is_contiguous():
+        raise ValueError("ffn_forward_host: q_host must be a contiguous bf16 CPU tensor")
+    d_model = q_host.shape[-1]
+    T = q_host.numel() // d_model if d_model else 0
+    _ffn_shapes(torch.empty(d_model, dtype=torch.bfloat16, device=K1.device), K1, K2, V)
+    d_ff, r = K1.shape
+    if out_host is None:
+        out_host = torch.empty(tuple(q_host.shape), dtype=torch.bfloat16, pin_memory=q_host.is_pinned())
+    elif out_host.device.type != "cpu" or out_host.dtype != torch.bfloat16 or out_host.shape != q_host.shape \
+            or not out_host.is_contiguous():
+        raise ValueError("ffn_forward_host: out_host must be a contiguous bf16 CPU tensor shaped like q_host")
+    rc = _binding.lib().spark_ffn_forward_host(q_host.data_ptr(), K1.data_ptr(), K2.data_ptr(), V.data_ptr(), T,
+                                               d_model, r, d_ff, int(k), out_host.data_ptr(),
+                                               _binding.stream_handle(stream))
+    _binding.check("spark_ffn_forward_host", rc)
+    return out_host
 
 
 def ffn_forward_debug(q, K1, K2, V, k: int, stream=None) -> dict:

@@ -29,7 +29,7 @@ EXPORTS = ("spark_ffn_forward", "spark_ffn_forward_tokens", "spark_ffn_forward_d
            "spark_set_wait_limit_ns", "spark_selftest_wait_timeout", "spark_version", "spark_ffn_forward_noalloc",
            "spark_ffn_decode_stack", "spark_set_weight_overlap", "spark_attention_decode",
            "spark_attention_decode_debug", "spark_ffn_predictor", "stat_topk_soft_threshold_causal",
-           "stat_topk_huber", "stat_topk_huber_backward", "spark_debug_violations")
+           "stat_topk_huber", "stat_topk_huber_backward", "spark_debug_violations", "spark_ffn_forward_host")
 
 _lock = threading.Lock()
 _lib = None
@@ -51,6 +51,7 @@ def _load(path: str) -> ctypes.CDLL:
     vp, ci = ctypes.c_void_p, ctypes.c_int
     L.spark_ffn_forward.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, vp, vp]
     L.spark_ffn_forward_tokens.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp]
+    L.spark_ffn_forward_host.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp]
     L.spark_ffn_forward_debug.argtypes = [vp, vp, vp, vp, ci, ci, ci, ci, ci, vp, vp, vp, vp, vp]
     L.stat_topk_soft_threshold.argtypes = [vp, ci, ci, ci, vp, vp]
     L.spark_query_status.argtypes = [vp]

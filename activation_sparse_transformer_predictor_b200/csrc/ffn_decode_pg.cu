@@ -27,6 +27,11 @@
 //  R  CTA b owns 16 output columns: it sums the partials of all slices in a
 //     fixed order and stores bf16 (stack mode: h_out = h + bf16(out)).
 // No atomics: results are bit-reproducible.
+//
+// With q and out in mapped (pinned) host memory, a one-CTA kernel F ahead of P
+// copies q into the workspace (P, launched programmatically behind F, streams
+// K1 meanwhile), and R stores out straight into host memory: no copy-engine
+// transfer sits between two calls' kernels.
 #include <map>
 #include <mutex>
 #include <utility>
@@ -482,6 +487,28 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
   }
 }
 
+// ------------------------------------------------------------------------ F
+// q from host memory (a device-visible address of a mapped pinned buffer) into
+// the device copy P reads.  It lets its dependent (P) launch at once, reads q,
+// and writes it only after the kernel ahead of it has completed, so that F's
+// completion also stands for that kernel's (the chain stays ordered).
+__global__ void __launch_bounds__(256) decode_fetch_q_kernel(const uint4* src, uint4* dst, int n16) {
+  griddep_launch_dependents();
+  constexpr int kPer = 4;  // up to 4 x 256 chunks of 16 bytes: d_model <= 8192
+  uint4 v[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = threadIdx.x + j * 256;
+    if (i < n16) v[j] = __ldcv(src + i);  // host memory: plain (coherent) loads, not the read-only path
+  }
+  griddep_wait();
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = threadIdx.x + j * 256;
+    if (i < n16) dst[i] = v[j];
+  }
+}
+
 // ------------------------------------------------------------------------ R
 // CTA b owns columns [16b, 16b + 16): thread t sums the partials of slices
 // t/4, t/4 + 32, ... for its float4 of columns (t % 4), then the 32 subsets are
@@ -645,6 +672,18 @@ cudaError_t launch_decode_pg(const DecodePgPlan& pl, const DecodePgArgs& a, cuda
   cudaLaunchConfig_t cfg = {};
   cfg.stream = stream;
   cfg.attrs = attr;
+  if (a.q_fetch != nullptr) {
+    // F: q from host memory; programmatic like P (it writes only after its wait)
+    const int n16 = a.d_model / 8;
+    if (a.d_model % 8 != 0 || n16 > 4 * 256 || a.h_in != nullptr) return cudaErrorInvalidValue;
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    cfg.numAttrs = a.overlap_weights ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, decode_fetch_q_kernel, static_cast<const uint4*>(a.q_fetch),
+                           reinterpret_cast<uint4*>(const_cast<void*>(a.q)), n16);
+    if (e != cudaSuccess) return e;
+  }
   // P: programmatic only with weight overlap (it reads K1 before its wait)
   cfg.gridDim = dim3(pl.n_slices);
   cfg.blockDim = dim3(kPThreads);

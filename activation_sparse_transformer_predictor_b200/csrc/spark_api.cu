@@ -43,6 +43,8 @@ struct Workspace {
 std::mutex g_mutex;
 std::map<int, DeviceInfo> g_devices;
 std::map<std::pair<int, cudaStream_t>, Workspace> g_workspaces;
+// device copies of q and out for spark_ffn_forward_host, per device and stream
+std::map<std::pair<int, cudaStream_t>, Workspace> g_staging;
 
 int current_device(int* dev) {
   return cudaGetDevice(dev) == cudaSuccess ? SPARK_OK : SPARK_ECUDA;
@@ -63,11 +65,13 @@ int device_info(int dev, DeviceInfo* out) {
   return di.is_sm100 ? SPARK_OK : SPARK_EDEVICE;
 }
 
-// Returns a workspace of at least `bytes` for (dev, stream).  A new or regrown
-// workspace starts with a zeroed device control block.
-int get_workspace(int dev, cudaStream_t stream, size_t bytes, void** ptr) {
+// Returns a buffer of `pool` of at least `bytes` for (dev, stream), allocated
+// or regrown on `stream` (never inside a stream capture).  With `zero_control`
+// a new buffer starts with a zeroed device control block.
+int get_buffer(std::map<std::pair<int, cudaStream_t>, Workspace>& pool, int dev, cudaStream_t stream, size_t bytes,
+               bool zero_control, void** ptr) {
   std::lock_guard<std::mutex> lock(g_mutex);
-  Workspace& ws = g_workspaces[{dev, stream}];
+  Workspace& ws = pool[{dev, stream}];
   if (ws.bytes >= bytes && ws.ptr != nullptr) {
     *ptr = ws.ptr;
     return SPARK_OK;
@@ -86,14 +90,32 @@ int get_workspace(int dev, cudaStream_t stream, size_t bytes, void** ptr) {
     cudaGetLastError();
     return SPARK_ENOMEM;
   }
-  if (cudaMemsetAsync(p, 0, sizeof(DeviceControl), stream) != cudaSuccess) return SPARK_ECUDA;
+  if (zero_control && cudaMemsetAsync(p, 0, sizeof(DeviceControl), stream) != cudaSuccess) return SPARK_ECUDA;
   ws.ptr = p;
   ws.bytes = want;
   *ptr = p;
   return SPARK_OK;
 }
 
+// The kernels' workspace for (dev, stream): control block first, then scratch.
+int get_workspace(int dev, cudaStream_t stream, size_t bytes, void** ptr) {
+  return get_buffer(g_workspaces, dev, stream, bytes, true, ptr);
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The device-visible address of host memory p, if p lies in a pinned buffer
+// that is mapped for device `dev` (cudaHostAlloc / cudaHostRegister with
+// mapping, which unified addressing implies); else nullptr.
+void* mapped_host_address(const void* p, int dev) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (at.type != cudaMemoryTypeHost || at.device != dev) return nullptr;
+  return at.devicePointer;
+}
 
 bool overlaps(const void* a, size_t abytes, const void* b, size_t bbytes) {
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
@@ -139,9 +161,11 @@ int check_ffn_args(const void* q, const void* K1, const void* K2, const void* V,
   return SPARK_OK;
 }
 
+// q_fetch (single-token decode only): a device-visible address of q in mapped
+// host memory, copied to q (a device buffer) by the first kernel of the call.
 int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* V, int T, int d_model, int r,
                      int d_ff, int k, void* out, float* x_out, float* theta_out, unsigned char* active_out,
-                     cudaStream_t stream, int never_arrive) {
+                     cudaStream_t stream, int never_arrive, const void* q_fetch = nullptr) {
   int dev;
   if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
   DeviceInfo di;
@@ -185,6 +209,7 @@ int ffn_forward_impl(const void* q, const void* K1, const void* K2, const void* 
       if (wst != SPARK_OK) return wst;
       DecodePgArgs a;
       a.q = q;
+      a.q_fetch = q_fetch;
       a.K1 = K1;
       a.K2 = K2;
       a.V = V;
@@ -281,6 +306,51 @@ SPARK_API int spark_ffn_forward_debug(const void* q, const void* K1, const void*
   if (x_out != nullptr && !aligned16(x_out)) return SPARK_EALIGN;
   return ffn_forward_impl(q, K1, K2, V, n_tokens, d_model, r, d_ff, k, out, x_out, theta_out, active_out,
                           reinterpret_cast<cudaStream_t>(stream), 0);
+}
+
+SPARK_API int spark_ffn_forward_host(const void* q_host, const void* K1, const void* K2, const void* V,
+                                     int n_tokens, int d_model, int r, int d_ff, int k, void* out_host,
+                                     spark_stream_t stream_) {
+  if (n_tokens == 0) return SPARK_OK;
+  // every check spark_ffn_forward_tokens makes, before anything is enqueued
+  if (!q_host || !out_host || !K1 || !K2 || !V) return SPARK_EINVAL;
+  if (n_tokens < 1 || d_model < 2 || !(r > 0 && r < d_model) || !(k > 0 && k < d_ff)) return SPARK_EINVAL;
+  if (r % 8 != 0 || d_model % 8 != 0) return SPARK_EALIGN;
+  if (!aligned16(K1) || !aligned16(K2) || !aligned16(V)) return SPARK_EALIGN;
+  const size_t bytes = static_cast<size_t>(n_tokens) * d_model * 2;
+  if (overlaps(q_host, bytes, out_host, bytes)) return SPARK_EINVAL;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  int dev;
+  if (current_device(&dev) != SPARK_OK) return SPARK_ECUDA;
+  DeviceInfo di;
+  const int dst = device_info(dev, &di);
+  if (dst != SPARK_OK) return dst;
+  const size_t half = (bytes + 255) / 256 * 256;
+  void* st = nullptr;
+  const int wst = get_buffer(g_staging, dev, stream, 2 * half, false, &st);
+  if (wst != SPARK_OK) return wst;
+  void* qd = st;
+  void* od = static_cast<unsigned char*>(st) + half;
+  if (n_tokens == 1 && plan_decode_pg(d_model, r, d_ff, di.num_sms, di.smem_optin).ok) {
+    // single-token decode from mapped pinned buffers: the first kernel reads q
+    // from host memory and the last one stores out into it (no copy-engine
+    // transfers between calls)
+    void* qm = aligned16(q_host) ? mapped_host_address(q_host, dev) : nullptr;
+    void* om = qm != nullptr ? mapped_host_address(out_host, dev) : nullptr;
+    if (qm != nullptr && om != nullptr)
+      return ffn_forward_impl(qd, K1, K2, V, 1, d_model, r, d_ff, k, om, nullptr, nullptr, nullptr, stream, 0, qm);
+  }
+  if (cudaMemcpyAsync(qd, q_host, bytes, cudaMemcpyHostToDevice, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  const int rc = spark_ffn_forward_tokens(qd, K1, K2, V, n_tokens, d_model, r, d_ff, k, od, stream_);
+  if (rc != SPARK_OK) return rc;
+  if (cudaMemcpyAsync(out_host, od, bytes, cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
+    cudaGetLastError();
+    return SPARK_ECUDA;
+  }
+  return SPARK_OK;
 }
 
 SPARK_API int spark_ffn_predictor(const void* q, const void* K1, int n_tokens, int d_model, int r, int d_ff,
@@ -564,12 +634,14 @@ SPARK_API int spark_release_workspace(void) {
   int prev = 0;
   cudaGetDevice(&prev);
   int rc = SPARK_OK;
-  for (auto& kv : g_workspaces) {
-    if (kv.second.ptr == nullptr) continue;
-    cudaSetDevice(kv.first.first);
-    if (cudaDeviceSynchronize() != cudaSuccess || cudaFree(kv.second.ptr) != cudaSuccess) rc = SPARK_ECUDA;
+  for (auto* pool : {&g_workspaces, &g_staging}) {
+    for (auto& kv : *pool) {
+      if (kv.second.ptr == nullptr) continue;
+      cudaSetDevice(kv.first.first);
+      if (cudaDeviceSynchronize() != cudaSuccess || cudaFree(kv.second.ptr) != cudaSuccess) rc = SPARK_ECUDA;
+    }
+    pool->clear();
   }
-  g_workspaces.clear();
   cudaSetDevice(prev);
   return rc;
 }

@@ -94,11 +94,15 @@ DecodePgPlan plan_decode_pg(int d_model, int r, int d_ff, int num_sms, size_t sm
 
 struct DecodePgArgs {
   const void* q = nullptr;      // bf16 [d_model] (ignored when h_in is set)
+  // Device-visible address of q in mapped host memory, or nullptr: a one-CTA
+  // kernel first copies it to q (then a device buffer the call may write).
+  const void* q_fetch = nullptr;
   const float* h_in = nullptr;  // stack mode: q = bf16(RMSNorm(h_in)), formed by the score kernel
   const void* K1 = nullptr;
   const void* K2 = nullptr;
   const void* V = nullptr;
-  void* out = nullptr;          // bf16 [d_model]; may be nullptr in stack mode
+  void* out = nullptr;          // bf16 [d_model] (device memory or a device-visible address of mapped
+                                // host memory); may be nullptr in stack mode
   int d_model = 0, r = 0, d_ff = 0;
   float Q = 0.f;
   float eps = 0.f;

@@ -100,6 +100,29 @@ SPARK_API int spark_ffn_forward_tokens(const void* q, const void* K1, const void
                                        int k, void* out, spark_stream_t stream);
 
 /*
+ * spark_ffn_forward_tokens with q and out in HOST memory: copies q (bf16
+ * [n_tokens][d_model]) to a device buffer, runs the forward, and copies out
+ * back, all enqueued on `stream` (one H2D copy, the kernels, one D2H copy).
+ * The weights are device pointers as above.  Like any asynchronous copy, q_host
+ * must stay unchanged, and out_host unread, until the stream has passed the
+ * call: synchronise the stream before reading out_host.  For the call to be
+ * asynchronous the host buffers must be pinned (cudaHostAlloc /
+ * cudaHostRegister); with pageable memory the CUDA runtime stages them and the
+ * call returns only after the output copy has completed.  For one token, with
+ * both buffers pinned and mapped for the current device (as unified addressing
+ * makes them) and q_host 16-byte aligned, no copy engine is used: the call's
+ * first kernel reads q from host memory and its last kernel stores out there.  The device buffers
+ * (2 n_tokens d_model bf16) belong to the library, one pair per device and
+ * stream, grown like the workspace (so not inside a stream capture) and freed
+ * by spark_release_workspace.  Same argument checks and errors as
+ * spark_ffn_forward_tokens (q_host and out_host need no alignment but may not
+ * overlap), all made before anything is enqueued.
+ */
+SPARK_API int spark_ffn_forward_host(const void* q_host, const void* K1, const void* K2, const void* V,
+                                     int n_tokens, int d_model, int r, int d_ff, int k, void* out_host,
+                                     spark_stream_t stream);
+
+/*
  * spark_ffn_forward_tokens that also returns the intermediate values it used,
  * for parity checks.  Each extra output may be NULL:
  *   x_out      : fp32 [n_tokens][d_ff]   predictor scores x (16-byte aligned, else SPARK_EALIGN)

@@ -241,3 +241,45 @@ def test_decode_weight_overlap_in_graph_is_bit_identical():
     finally:
         spark.set_weight_overlap(False)
     assert spark.query_status() == 0
+
+
+@pytest.mark.parametrize("shape,T", [(GEMMA, 1), (TINY, 4), (GEMMA, 100)])
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_buffers_give_the_device_entry_points_bits(shape, T, pinned):
+    """spark_ffn_forward_host (q in and out back through host memory) on two calls in a row on one
+    stream (its device copies of q and out are reused) against the device-pointer entry point."""
+    d_model, r, d_ff, k = shape
+    for layer in (90 + T, 91 + T):
+        dev, _ = make_layer(d_model, r, d_ff, T, layer=layer)
+        q = dev["q"] if T > 1 else dev["q"][0]
+        ref = spark.ffn_forward(q, dev["K1"], dev["K2"], dev["V"], k)
+        qh = q.cpu()
+        if pinned:
+            qh = qh.pin_memory()
+        out = spark.ffn_forward_host(qh, dev["K1"], dev["K2"], dev["V"], k)
+        torch.cuda.synchronize()
+        assert spark.query_status() == 0
+        assert out.shape == qh.shape and torch.equal(out, ref.cpu())
+
+
+def test_host_buffers_in_a_decode_loop_with_weight_overlap():
+    """Single-token calls from mapped pinned buffers back to back with weight overlap on (the first
+    kernel of each call reads q from host memory while the next call's K1 streams), against the
+    device entry point, one layer per call."""
+    d_model, r, d_ff, k = GEMMA
+    layers = [make_layer(d_model, r, d_ff, 1, layer=120 + i) for i in range(3)]
+    refs = [spark.ffn_forward(dv["q"][0], dv["K1"], dv["K2"], dv["V"], k).cpu() for dv, _ in layers]
+    qh = [dv["q"][0].cpu().pin_memory() for dv, _ in layers]
+    oh = [torch.empty_like(q).pin_memory() for q in qh]
+    spark.set_weight_overlap(True)
+    try:
+        for rep in range(2):
+            for i, (dv, _) in enumerate(layers):
+                spark.ffn_forward_host(qh[i], dv["K1"], dv["K2"], dv["V"], k, out_host=oh[i])
+            torch.cuda.synchronize()
+            assert spark.query_status() == 0
+            for i in range(3):
+                assert torch.equal(oh[i], refs[i]), (rep, i)
+                oh[i].zero_()
+    finally:
+        spark.set_weight_overlap(False)

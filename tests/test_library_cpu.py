@@ -71,6 +71,16 @@ def test_argument_checks_before_any_device_work(L):
     assert f(vp((1 << 20) + 2), fake, fake, fake, 1, 64, 32, 256, 20, vp(1 << 30), null) == EALIGN
     # out overlapping q
     assert f(fake, vp(1 << 24), vp(1 << 25), vp(1 << 26), 1, 64, 32, 256, 20, vp((1 << 20) + 64), null) == EINVAL
+    hf = L.spark_ffn_forward_host  # host q / out: no alignment asked of them, weights as above
+    assert hf(fake, fake, fake, fake, 0, 64, 32, 256, 20, vp(1 << 30), null) == 0  # empty batch: no-op
+    assert hf(null, fake, fake, fake, 1, 64, 32, 256, 20, vp(1 << 30), null) == EINVAL  # NULL q_host
+    assert hf(fake, fake, fake, fake, 1, 64, 32, 256, 20, null, null) == EINVAL  # NULL out_host
+    assert hf(fake, null, fake, fake, 1, 64, 32, 256, 20, vp(1 << 30), null) == EINVAL  # NULL K1
+    assert hf(fake, fake, fake, fake, -1, 64, 32, 256, 20, vp(1 << 30), null) == EINVAL  # T < 0
+    assert hf(fake, fake, fake, fake, 1, 64, 32, 256, 256, vp(1 << 30), null) == EINVAL  # k == d_ff
+    assert hf(fake, fake, fake, fake, 1, 64, 36, 256, 20, vp(1 << 30), null) == EALIGN  # r % 8
+    assert hf(fake, vp((1 << 20) + 2), fake, fake, 1, 64, 32, 256, 20, vp(1 << 30), null) == EALIGN  # K1
+    assert hf(fake, fake, fake, fake, 2, 64, 32, 256, 20, vp((1 << 20) + 2), null) == EINVAL  # out on q
     t = L.stat_topk_soft_threshold
     assert t(fake, 4, 100, 0, fake, null) == EINVAL
     assert t(fake, 4, 100, 100, fake, null) == EINVAL
