@@ -31,7 +31,9 @@
 // warp 1 = TMEM allocator and single-thread tcgen05.mma issuer (M 128, N 128 or
 // 256, K 16 per instruction, fp32 accumulators in TMEM, two accumulators so
 // that the epilogue of one tile overlaps the main loop of the next), the
-// remaining warps = epilogue (tcgen05.ld, 32 TMEM lanes per warp).  Every wait
+// remaining warps = epilogue (tcgen05.ld, 32 TMEM lanes per warp).  A unit is
+// 128 tokens x 128 columns, x 256 once there are enough to fill the SMs, or x 64
+// for GEMMs 1 and 2 with a single token band (more CTAs streaming the weights).  Every wait
 // is bounded.  Each GEMM is launched as a programmatic dependent of the kernel
 // before it: barrier set-up and the TMEM allocation overlap that kernel's tail,
 // and nothing touches global memory before griddepcontrol.wait (measured
@@ -73,7 +75,8 @@ struct GemmParams {
   float4* Xt;             // predictor scores in 128 x 128 tiles: written by GEMM 1, read by GEMM 2
   int xt_tiles_n;         // 128-column tiles per 128-row band of Xt
   float2* moments;        // [M][mom_stride] (mean, M2) of each 128-neuron tile
-  int mom_stride;         // 128-neuron tiles per row of moments
+  int mom_stride;         // neuron tiles per row of moments
+  int mom_w;              // neurons per moments tile: 128, or 64 with 64-column units
   const float* theta;     // [M] thresholds from theta_kernel, or nullptr: GEMM 2's epilogue derives them
   float Q;                // standard-normal quantile Q(1 - k/d_ff) of the threshold
   float* theta_out;       // optional [M]: the thresholds GEMM 2 derived (debug entry point)
@@ -261,7 +264,7 @@ __device__ __forceinline__ float gate_theta(const GemmParams& p, int m, int row,
     for (int u = 0; u < kB; ++u) mm[u] = (ok && jb + u < j1) ? mr[jb + u] : make_float2(0.f, 0.f);
 #pragma unroll
     for (int u = 0; u < kB; ++u)
-      if (jb + u < j1) s = fmaf(static_cast<float>(min(BN, p.N - (jb + u) * BN)), mm[u].x, s);
+      if (jb + u < j1) s = fmaf(static_cast<float>(min(p.mom_w, p.N - (jb + u) * p.mom_w)), mm[u].x, s);
   }
   tred[colgrp * BM + row] = s;
   named_bar_sync(1 + quarter, 128);
@@ -275,7 +278,7 @@ __device__ __forceinline__ float gate_theta(const GemmParams& p, int m, int row,
     for (int u = 0; u < kB; ++u)
       if (jb + u < j1) {
         const float d = mm[u].x - mean;
-        m2 += mm[u].y + static_cast<float>(min(BN, p.N - (jb + u) * BN)) * d * d;
+        m2 += mm[u].y + static_cast<float>(min(p.mom_w, p.N - (jb + u) * p.mom_w)) * d * d;
       }
   }
   tred[(4 + colgrp) * BM + row] = m2;
@@ -293,7 +296,11 @@ __device__ __forceinline__ float gate_theta(const GemmParams& p, int m, int row,
 // bytes, which only ever reach accumulator rows >= 64 -- rows no token owns,
 // which the epilogue skips.  The 24 KB stages let 8 of them (128 KB of weights)
 // be in flight instead of 6 (96 KB).
-template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false, bool A64 = false>
+// NW (GEMMs 1 and 2, one 128-token band): a unit is 128 rows x 64 columns, so
+// that twice as many CTAs stream the weights when there are only 72 128-column
+// tiles; its scores fill half of a 128 x 128 score tile and its moments cover
+// 64 neurons.
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false, bool A64 = false, bool NW = false>
 __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     umma_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA2,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB2,
@@ -301,10 +308,14 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   static_assert(!WIDE || B_NMAJOR == (EPI == kEpiOut), "wide GEMM 3 takes V N-major; GEMMs 1 and 2 K-major");
   static_assert(!DUAL || EPI == kEpiOut, "two A operands (h_hi, h_lo) are GEMM 3's");
   static_assert(!A64 || (EPI != kEpiOut && !WIDE), "64-row A boxes: narrow GEMMs 1 and 2 only");
+  static_assert(!NW || (!WIDE && EPI != kEpiOut), "64-column units: GEMMs 1 and 2 only");
   constexpr int kBTiles = WIDE ? 2 : 1;
+  constexpr int kUC = WIDE ? 2 * BN : (NW ? BN / 2 : BN);  // columns of one unit
+  constexpr int kHalf = WIDE ? BN : kUC;                     // columns per B tile
+  constexpr int kBB = kHalf * BK * 2;                        // bytes of one K-major B tile
   constexpr int kAB = A64 ? kABytes / 2 : kABytes;  // bytes of one stage's A box
-  constexpr int kStageBytes = kAB * (DUAL ? 2 : 1) + kBBytes * kBTiles;
-  constexpr int kAccCols = WIDE ? 2 * BN : BN;  // TMEM columns of one tile's accumulators
+  constexpr int kStageBytes = kAB * (DUAL ? 2 : 1) + (EPI == kEpiOut ? kBBytes : kBB) * kBTiles;
+  constexpr int kAccCols = kUC;  // TMEM columns of one tile's accumulators
   constexpr int kTmemCols = 2 * kAccCols;       // double buffered
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -359,8 +370,10 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         // the gate epilogue reads this unit's score tiles a whole main loop from
         // now: pull them into L2 (a 64 KB tile is contiguous)
 #pragma unroll
-        for (int h = 0; h < kBTiles; ++h)
-          if ((tn * kBTiles + h) * BN < p.N) prefetch_l2_bulk(xt_tile(p, tm, (tn * kBTiles + h) * BN), BM * BN * 4);
+        for (int h = 0; h < kBTiles; ++h) {
+          const int cb = tn * kUC + h * BN;  // a 64-column unit's scores are half of a tile
+          if (cb < p.N) prefetch_l2_bulk(xt_tile(p, tm, cb) + cb % BN / 4 * BM, BM * kHalf * 4);
+        }
       }
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait_bounded(&empty[stage], ph ^ 1u, p.wait_limit_ns, ctl, 100) || *abort_flag) {
@@ -389,7 +402,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         } else {
 #pragma unroll
           for (int h = 0; h < kBTiles; ++h)
-            tma_load_2d(sb + h * kBBytes, &tmB, kb * BK, (tn * kBTiles + h) * BN, &full[stage]);
+            tma_load_2d(sb + h * kBB, &tmB, kb * BK, tn * kUC + h * BN, &full[stage]);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -424,7 +437,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     // ------------------------------------------------------------ MMA issuer
     // a wide unit is one M 128 x N 256 instruction per K 16 step: its two B tiles
     // are adjacent in shared memory, 8-row atoms 1024 B apart throughout
-    constexpr uint32_t idesc = make_idesc(B_NMAJOR, WIDE ? 2 * BN : BN);
+    constexpr uint32_t idesc = make_idesc(B_NMAJOR, kUC);
     int stage = 0;
     uint32_t ph = 0;
     uint32_t uses[2] = {0u, 0u};
@@ -481,15 +494,15 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       int tm, tn, kb0, kb1;
       decode_unit<EPI>(p, unit, tm, tn, kb0, kb1);
       const int m = tm * BM + row;
-      const int n_base = tn * BN * kBTiles;
+      const int n_base = tn * kUC;
       const bool row_ok = m < p.M;
       // GEMM 2: this warp's columns of the tile (a wide unit's half, or half of a
       // narrow unit) and this row's scores there, stored by GEMM 1, loaded while
       // the accumulator is still being formed
-      constexpr int kGateCols = (WIDE ? 2 * BN : BN) / (epi_warps(kEpiGate) / 4);
+      constexpr int kGateCols = kUC / (epi_warps(kEpiGate) / 4);
       const int gcol = colgrp * kGateCols;                // first column within the unit
-      const int gtile_nb = n_base + gcol / BN * BN;       // first column of its score tile
-      const int gx0 = gcol % BN / 4;                      // its first float4 group in that tile
+      const int gtile_nb = (n_base + gcol) / BN * BN;     // first column of its score tile
+      const int gx0 = (n_base + gcol) % BN / 4;           // its first float4 group in that tile
       float4 xr[EPI == kEpiGate ? kGateCols / 4 : 1];
       float th = 0.f;
       if (EPI == kEpiGate) {
@@ -519,10 +532,11 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           const int nb = n_base + h * BN;
           const uint32_t ta = taddr + static_cast<uint32_t>(h * BN);
           float4* xt = xt_tile(p, tm, nb);
+          const int g0 = nb % BN / 4;  // first float4 group of these columns in their tile
           float sum = 0.f;
           int cnt = 0;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = 0; c < kHalf; c += 32) {
             float w[32];
             tmem_ld32(ta + c, w);
 #pragma unroll
@@ -538,7 +552,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
               if (row_ok && n < p.N && p.Xt != nullptr && SPARK_CHECK(tm < p.tiles_m && nb / BN < p.xt_tiles_n)) {
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
-                  xt[((c + s) / 4 + q4) * BM + row] =
+                  xt[(g0 + (c + s) / 4 + q4) * BM + row] =
                       make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
               }
               if (p.X != nullptr) {
@@ -576,7 +590,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
           const float mean = cnt > 0 ? sum / static_cast<float>(cnt) : 0.f;
           float m2 = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
+          for (int c = 0; c < kHalf; c += 32) {
             float w[32];
             tmem_ld32(ta + c, w);
             const int n = nb + c;
@@ -587,7 +601,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                 m2 += d * d;
               }
           }
-          if (row_ok && nb < p.N) p.moments[static_cast<size_t>(m) * p.mom_stride + nb / BN] = make_float2(mean, m2);
+          if (row_ok && nb < p.N) p.moments[static_cast<size_t>(m) * p.mom_stride + nb / p.mom_w] = make_float2(mean, m2);
         }
       } else if (EPI == kEpiGate) {
         {
@@ -703,22 +717,22 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
 
 // theta per token from the tile moments: two passes over the partials
 // (weighted mean, then M2 = sum M2_j + n_j (mean_j - mean)^2), fixed order.
-__global__ void __launch_bounds__(128) theta_kernel(const float2* moments, int M, int N, int tiles_n, float Q,
-                                                    float* theta, float* theta_out) {
+__global__ void __launch_bounds__(128) theta_kernel(const float2* moments, int M, int N, int tiles_n, int mw,
+                                                    float Q, float* theta, float* theta_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.x * 4 + warp;
   if (m >= M) return;
   const float2* mr = moments + static_cast<size_t>(m) * tiles_n;
   float s = 0.f;
   for (int j = lane; j < tiles_n; j += 32) {
-    const float nj = static_cast<float>(min(BN, N - j * BN));
+    const float nj = static_cast<float>(min(mw, N - j * mw));
     s = fmaf(nj, mr[j].x, s);
   }
   s = __shfl_sync(0xffffffffu, warp_sum(s), 0);
   const float mean = s / static_cast<float>(N);
   float m2 = 0.f;
   for (int j = lane; j < tiles_n; j += 32) {
-    const float nj = static_cast<float>(min(BN, N - j * BN));
+    const float nj = static_cast<float>(min(mw, N - j * mw));
     const float d = mr[j].x - mean;
     m2 += mr[j].y + nj * d * d;
   }
@@ -780,13 +794,13 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false, bool A64 = false>
+template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false, bool A64 = false, bool NW = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const CUtensorMap& b2,
                         const GemmParams& p, int num_sms, cudaStream_t stream) {
-  constexpr int kStageBytes = (A64 ? kABytes / 2 : kABytes) * (DUAL ? 2 : 1) + kBBytes * (WIDE ? 2 : 1);
+  constexpr int kStageBytes = (A64 ? kABytes / 2 : kABytes) * (DUAL ? 2 : 1) + (NW ? kBBytes / 2 : kBBytes) * (WIDE ? 2 : 1);
   constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256 + (EPI == kEpiGate ? 8 * BM * 4 : 0) +
                           (EPI == kEpiPredictor ? 4 * 2048 : 0);
-  auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE, A64>;
+  auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE, A64, NW>;
   static int set_dev = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -818,7 +832,7 @@ size_t predictor_workspace_bytes(int, int) { return align256(sizeof(DeviceContro
 size_t prefill_workspace_bytes(int T, int d_model, int d_ff, int num_sms) {
   const int tiles_n = (d_ff + BN - 1) / BN;
   size_t b = align256(sizeof(DeviceControl));
-  b += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));            // moments
+  b += align256(static_cast<size_t>(T) * ((d_ff + 63) / 64) * sizeof(float2));  // moments (64-neuron tiles at most)
   b += align256(static_cast<size_t>(T) * 4);                                   // theta
   b += 2 * static_cast<size_t>((T + BM - 1) / BM) * ((d_ff + BK - 1) / BK) * BM * BK * 2;  // h_hi, h_lo
   b += static_cast<size_t>((T + BM - 1) / BM) * tiles_n * BM * BN * 4;         // tiled scores
@@ -851,7 +865,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   unsigned char* ws = static_cast<unsigned char*>(a.workspace);
   size_t off = align256(sizeof(DeviceControl));
   float2* moments = reinterpret_cast<float2*>(ws + off);
-  off += align256(static_cast<size_t>(T) * tiles_n * sizeof(float2));
+  off += align256(static_cast<size_t>(T) * ((d_ff + 63) / 64) * sizeof(float2));
   float* theta = reinterpret_cast<float*>(ws + off);
   off += align256(static_cast<size_t>(T) * 4);
   const int h_kb = (d_ff + BK - 1) / BK;
@@ -876,6 +890,18 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
       !make_tmap(&tk2, a.K2, d2, d_ff, static_cast<uint64_t>(d2) * 2, BK, BN) ||
       !make_tmap(&tv, a.V, d_model, d_ff, static_cast<uint64_t>(d_model) * 2, 64, BK))
     return cudaErrorInvalidValue;
+  // 65 to 128 tokens (one band): GEMMs 1 and 2 run 128 x 64 units (64-row weight
+  // boxes), so that 144 CTAs rather than 72 stream the weights (T = 100 47.6 ->
+  // 45.2 us, T = 128 49.2 -> 46.8).  Up to 64 tokens they measured no faster
+  // (T = 64 43.8 -> 45.3 us: GEMM 2's epilogue warps then merge the moments of
+  // twice as many tiles per CTA, in twice as many CTAs, while a shorter main loop
+  // hides less of it).
+  const bool nw = T > 64 && T <= BM;
+  const int nw_tiles = (d_ff + 63) / 64;
+  CUtensorMap tk1n, tk2n;
+  if (nw && (!make_tmap(&tk1n, a.K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, 64) ||
+             !make_tmap(&tk2n, a.K2, d2, d_ff, static_cast<uint64_t>(d2) * 2, BK, 64)))
+    return cudaErrorInvalidValue;
 
   GemmParams g{};
   g.ctl = reinterpret_cast<DeviceControl*>(ws);
@@ -884,7 +910,8 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   g.Xt = Xt;      // GEMM 1 stores the scores once, tiled; GEMM 2's gate reads them back
   g.xt_tiles_n = tiles_n;
   g.moments = moments;
-  g.mom_stride = tiles_n;
+  g.mom_stride = nw ? nw_tiles : tiles_n;
+  g.mom_w = nw ? 64 : BN;
   g.theta = nullptr;
   g.Q = a.Q;
   g.theta_out = a.theta_out;
@@ -913,6 +940,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
     g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
     g.units = wide_units;
     e = launch_gemm<kEpiPredictor, false, false, 4, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  } else if (nw) {
+    g.tiles_n = nw_tiles;
+    g.units = g.tiles_m * g.tiles_n;
+    e = launch_gemm<kEpiPredictor, false, false, 8, false, false, true>(tq1, tq1, tk1n, tk1n, g, num_sms, stream);
   } else if (a64) {
     e = launch_gemm<kEpiPredictor, false, false, 8, false, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
   } else {
@@ -927,9 +958,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   // CTA of a token band repeats that merge for the same rows, which at T = 256
   // (72 CTAs per band, 256 rows) cost more than it saved (+6 us), and with several
   // units per CTA it would sit between units: there theta_kernel runs first.
-  const int gate_units = wide_units >= num_sms ? wide_units : g.tiles_m * tiles_n;
+  const int gate_units = wide_units >= num_sms ? wide_units : g.tiles_m * (nw ? nw_tiles : tiles_n);
   if (T > 64 || wide_units >= num_sms || gate_units > num_sms) {
-    theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, tiles_n, a.Q, theta, a.theta_out);
+    theta_kernel<<<(T + 3) / 4, 128, 0, stream>>>(moments, T, d_ff, g.mom_stride, g.mom_w, a.Q, theta,
+                                                  a.theta_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     g.theta = theta;
   }
@@ -940,6 +972,10 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
     g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
     g.units = wide_units;
     e = launch_gemm<kEpiGate, false, false, 4, true>(tq2, tq2, tk2, tk2, g, num_sms, stream);
+  } else if (nw) {
+    g.tiles_n = nw_tiles;
+    g.units = g.tiles_m * g.tiles_n;
+    e = launch_gemm<kEpiGate, false, false, 8, false, false, true>(tq2, tq2, tk2n, tk2n, g, num_sms, stream);
   } else {
     g.tiles_n = tiles_n;
     g.units = g.tiles_m * g.tiles_n;
@@ -990,6 +1026,7 @@ cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, 
   g.xt_tiles_n = tiles_n;
   g.moments = nullptr;  // x only
   g.mom_stride = tiles_n;
+  g.mom_w = BN;
   g.M = T;
   g.N = d_ff;
   g.K = r;
@@ -1004,6 +1041,16 @@ cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, 
     g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
     g.units = wide_units;
     return launch_gemm<kEpiPredictor, false, false, 4, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  }
+  if (T <= BM) {
+    // one token band: 128 x 64 units, 144 CTAs streaming K1 (T = 16 10.8 -> 9.9 us,
+    // T = 128 11.7 -> 10.4)
+    CUtensorMap tk1n;
+    if (!make_tmap(&tk1n, K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, 64)) return cudaErrorInvalidValue;
+    g.tiles_n = (d_ff + 63) / 64;
+    g.units = g.tiles_m * g.tiles_n;
+    return a64 ? launch_gemm<kEpiPredictor, false, false, 12, false, true, true>(tq1, tq1, tk1n, tk1n, g, num_sms, stream)
+               : launch_gemm<kEpiPredictor, false, false, 8, false, false, true>(tq1, tq1, tk1n, tk1n, g, num_sms, stream);
   }
   if (a64) return launch_gemm<kEpiPredictor, false, false, 8, false, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
   return launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);

@@ -18,7 +18,9 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("shape,T", [
     ((2304, 1152, 9216, 737), 1),
+    ((2304, 1152, 9216, 737), 16),      # one token band: 128 x 64 units, 64-row token boxes
     ((2304, 1152, 9216, 737), 64),
+    ((2304, 1152, 9216, 737), 100),     # one token band: 128 x 64 units, 128-row token boxes
     ((2304, 1152, 9216, 737), 200),
     ((2304, 1152, 9216, 737), 1100),     # 128 x 256 units, ragged last token band
     ((264, 136, 1008, 80), 7),          # ragged r (two partial K blocks) and d_ff
@@ -36,9 +38,10 @@ def test_predictor_matches_oracle_scores(shape, T):
     assert np.all(np.abs(gx - orc["x"]) <= tol)
 
 
-def test_predictor_equals_the_prefill_scores():
+@pytest.mark.parametrize("T", [100, 256])
+def test_predictor_equals_the_prefill_scores(T):
     """The same GEMM as the predictor stage of spark_ffn_forward_debug: identical bits."""
-    d_model, r, d_ff, k, T = 2304, 1152, 9216, 737, 256
+    d_model, r, d_ff, k = 2304, 1152, 9216, 737
     dev, _ = make_layer(d_model, r, d_ff, T, layer=3)
     x = spark.ffn_predictor(dev["q"], dev["K1"])
     res = spark.ffn_forward_debug(dev["q"], dev["K1"], dev["K2"], dev["V"], k)
