@@ -60,8 +60,11 @@ constexpr int BK = 64;
 // warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; the rest: epilogue.
 // GEMM 2's gate epilogue (GELU, split, score loads: a chain of dependent
 // latencies per element) runs sixteen epilogue warps, four per TMEM lane
-// quarter, each on its own quarter of the unit's columns; the others run four.
-__host__ __device__ constexpr int epi_warps(int epi) { return epi == 2 ? 16 : 4; }
+// quarter, each on its own quarter of the unit's columns; GEMM 1's runs eight,
+// two per quarter, each on half of the columns (its score stores were the
+// longest phase of a one-unit launch: the predictor alone at T = 256 11.9 ->
+// 10.9 us together with 128-byte store rows); GEMM 3's runs four.
+__host__ __device__ constexpr int epi_warps(int epi) { return epi == 2 ? 16 : epi == 1 ? 8 : 4; }
 __host__ __device__ constexpr int gemm_threads(int epi) { return 64 + 32 * epi_warps(epi); }
 constexpr int kABytes = BM * BK * 2;  // 16 KB
 constexpr int kBBytes = BN * BK * 2;  // 16 KB
@@ -525,75 +528,78 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(acc * kAccCols);
       float v[16];
       if (EPI == kEpiPredictor) {
+        // two warps per TMEM lane quarter, each on half of the unit's columns: a
+        // wide unit's 128-column tile each, else half of the unit's one moments
+        // tile (the two halves' sums and M2 are combined through shared memory)
+        constexpr int kEpiCols = kUC / 2;
+        const int col0 = colgrp * kEpiCols;                 // first unit column of this warp
+        const int tile0 = WIDE ? n_base + col0 : n_base;    // first column of its moments tile
+        float4* stg = reinterpret_cast<float4*>(smem + STAGES * kStageBytes + 256) + (warp - 2) * 256;
+        float* red = reinterpret_cast<float*>(smem + STAGES * kStageBytes + 256 + epi_warps(EPI) * 4096);
+        float sum = 0.f;
 #pragma unroll 1
-        for (int h = 0; h < kBTiles; ++h) {
-          // one 128-column half, 32 columns per TMEM load; its moments about its
-          // mean (a second pass over TMEM) unless moments are not wanted
-          const int nb = n_base + h * BN;
-          const uint32_t ta = taddr + static_cast<uint32_t>(h * BN);
-          float4* xt = xt_tile(p, tm, nb);
-          const int g0 = nb % BN / 4;  // first float4 group of these columns in their tile
-          float sum = 0.f;
-          int cnt = 0;
-#pragma unroll 1
-          for (int c = 0; c < kHalf; c += 32) {
-            float w[32];
-            tmem_ld32(ta + c, w);
+        for (int c = col0; c < col0 + kEpiCols; c += 32) {
+          float w[32];
+          tmem_ld32(taddr + c, w);
+          const int nc0 = n_base + c;
+          if (p.X != nullptr) {
+            // through shared memory: lane l's 32 values go to row l of a 32 x 32
+            // staging block (16-byte chunks xor-swizzled by row), read back so that
+            // one store instruction covers 4 rows x 128 contiguous bytes
 #pragma unroll
-            for (int s = 0; s < 32; s += 16) {
-              const float* v = w + s;
-              const int n = nb + c + s;
+            for (int q8 = 0; q8 < 8; ++q8)
+              stg[lane * 8 + (q8 ^ (lane & 7))] = make_float4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
+            __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 16; ++j)
-                if (n + j < p.N) {
-                  sum += v[j];
-                  ++cnt;
+            for (int i = 0; i < 8; ++i) {
+              const int rr = i * 4 + (lane >> 3), q8 = lane & 7;
+              const float4 val = stg[rr * 8 + (q8 ^ (rr & 7))];
+              const int mr = tm * BM + quarter * 32 + rr;
+              const int nc = nc0 + 4 * q8;
+              if (mr < p.M) {
+                float* dst = p.X + static_cast<size_t>(mr) * p.N + nc;
+                if (nc + 4 <= p.N) {
+                  *reinterpret_cast<float4*>(dst) = val;
+                } else {
+                  if (nc < p.N) dst[0] = val.x;
+                  if (nc + 1 < p.N) dst[1] = val.y;
+                  if (nc + 2 < p.N) dst[2] = val.z;
                 }
-              if (row_ok && n < p.N && p.Xt != nullptr && SPARK_CHECK(tm < p.tiles_m && nb / BN < p.xt_tiles_n)) {
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                  xt[(g0 + (c + s) / 4 + q4) * BM + row] =
-                      make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-              }
-              if (p.X != nullptr) {
-                // through shared memory: lane l's 16 values go to row l of a 32 x 16
-                // staging block (16-byte chunks xor-swizzled), read back so that one
-                // store instruction covers 8 rows x 64 contiguous bytes
-                float4* stg = reinterpret_cast<float4*>(smem + STAGES * kStageBytes + 256) + quarter * 128;
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                  stg[lane * 4 + (q4 ^ ((lane >> 1) & 3))] =
-                      make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
-                __syncwarp();
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int rr = i * 8 + (lane >> 2), q4 = lane & 3;
-                  const float4 val = stg[rr * 4 + (q4 ^ ((rr >> 1) & 3))];
-                  const int mr = tm * BM + quarter * 32 + rr;
-                  const int nc = n + 4 * q4;
-                  if (mr < p.M) {
-                    float* dst = p.X + static_cast<size_t>(mr) * p.N + nc;
-                    if (nc + 4 <= p.N) {
-                      *reinterpret_cast<float4*>(dst) = val;
-                    } else {
-                      if (nc < p.N) dst[0] = val.x;
-                      if (nc + 1 < p.N) dst[1] = val.y;
-                      if (nc + 2 < p.N) dst[2] = val.z;
-                    }
-                  }
-                }
-                __syncwarp();
               }
             }
+            __syncwarp();
           }
-          if (p.moments == nullptr) continue;
+#pragma unroll
+          for (int s = 0; s < 32; s += 16) {
+            const float* v = w + s;
+            const int n = nc0 + s;
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (n + j < p.N) sum += v[j];
+            if (row_ok && n < p.N && p.Xt != nullptr && SPARK_CHECK(tm < p.tiles_m && n / BN < p.xt_tiles_n)) {
+              float4* xt = xt_tile(p, tm, n);
+              const int g0 = n % BN / 4;
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+                xt[(g0 + q4) * BM + row] = make_float4(v[4 * q4], v[4 * q4 + 1], v[4 * q4 + 2], v[4 * q4 + 3]);
+            }
+          }
+        }
+        if (p.moments != nullptr) {
+          const int tw = WIDE ? BN : p.mom_w;  // columns of a moments tile
+          const int cnt = tile0 < p.N ? min(tw, p.N - tile0) : 0;
+          if (!WIDE) {
+            red[colgrp * BM + row] = sum;
+            named_bar_sync(1 + quarter, 64);
+            sum = red[row] + red[BM + row];
+          }
           const float mean = cnt > 0 ? sum / static_cast<float>(cnt) : 0.f;
           float m2 = 0.f;
 #pragma unroll 1
-          for (int c = 0; c < kHalf; c += 32) {
+          for (int c = col0; c < col0 + kEpiCols; c += 32) {
             float w[32];
-            tmem_ld32(ta + c, w);
-            const int n = nb + c;
+            tmem_ld32(taddr + c, w);
+            const int n = n_base + c;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (n + j < p.N) {
@@ -601,7 +607,15 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
                 m2 += d * d;
               }
           }
-          if (row_ok && nb < p.N) p.moments[static_cast<size_t>(m) * p.mom_stride + nb / p.mom_w] = make_float2(mean, m2);
+          if (!WIDE) {
+            named_bar_sync(1 + quarter, 64);  // both halves' sums read before red is reused
+            red[colgrp * BM + row] = m2;
+            named_bar_sync(1 + quarter, 64);
+            m2 = red[row] + red[BM + row];
+            named_bar_sync(1 + quarter, 64);  // read before the next unit writes red
+          }
+          if (row_ok && tile0 < p.N && (WIDE || colgrp == 0))
+            p.moments[static_cast<size_t>(m) * p.mom_stride + tile0 / tw] = make_float2(mean, m2);
         }
       } else if (EPI == kEpiGate) {
         {
@@ -799,7 +813,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUten
                         const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int kStageBytes = (A64 ? kABytes / 2 : kABytes) * (DUAL ? 2 : 1) + (NW ? kBBytes / 2 : kBBytes) * (WIDE ? 2 : 1);
   constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256 + (EPI == kEpiGate ? 8 * BM * 4 : 0) +
-                          (EPI == kEpiPredictor ? 4 * 2048 : 0);
+                          (EPI == kEpiPredictor ? epi_warps(EPI) * 4096 + 2 * BM * 4 : 0);
   auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE, A64, NW>;
   static int set_dev = -1;
   int dev = 0;
