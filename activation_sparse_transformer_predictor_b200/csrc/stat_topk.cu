@@ -129,8 +129,8 @@ __global__ void __launch_bounds__(kTopkThreads) stat_topk_generic_kernel(const f
 // Masked entries are written as 0 and never used.  Q depends on n, so each CTA
 // evaluates it (double precision, Q(1 - p) = -Phi^-1(p) with CUDA's normcdfinv),
 // in one thread of its last warp while the row's loads are in flight.  The vector
-// kernel is held to 40 registers so that six 256-thread CTAs share an SM (165 us
-// instead of 188 for 32768 rows x 4096 on B200).
+// kernel is held to 32 registers so that eight 256-thread CTAs share an SM (32768
+// rows x 4096 on B200: 188 us at 48 registers, 165 at 40, 148 at 32).
 __device__ __forceinline__ int causal_visible(int row, int d, int n_q, int offset) {
   const long long pos = static_cast<long long>(offset) + row % n_q;
   return pos + 1 < d ? static_cast<int>(pos + 1) : d;
@@ -141,7 +141,7 @@ __device__ __forceinline__ float causal_quantile(int k, int n) {
 }
 
 template <int NV>
-__global__ void __launch_bounds__(kTopkThreads, 6) stat_topk_causal_vec_kernel(const float* x, float* out, int d, int k,
+__global__ void __launch_bounds__(kTopkThreads, 8) stat_topk_causal_vec_kernel(const float* x, float* out, int d, int k,
                                                                             int n_q, int offset, float* theta_out) {
   __shared__ Moments s_warp[kTopkWarps];
   __shared__ float s_theta, s_q;
