@@ -393,6 +393,10 @@ __global__ void __maxnreg__(128) decode_gather_kernel(const PgParams p) {
   __syncthreads();
   const int nact = misc_i[0];
   const float theta = misc_f[0];
+  // the K2 rows of the active neurons into L2 now, ahead of the next call's K1
+  // stream (released below once the V loads are issued): 13.45 -> 13.32 us per
+  // call with weight overlap, 15.19 -> 14.93 without
+  if (tid < nact) prefetch_l2_bulk(p.K2 + static_cast<size_t>(act_i[tid]) * p.d2, static_cast<unsigned>(p.d2) * 2);
   if (nact == 0) griddep_launch_dependents();
   if (c == 0 && tid == 0 && p.theta_out != nullptr) p.theta_out[0] = theta;
   if (p.active_out != nullptr)
