@@ -38,7 +38,10 @@
 // before it: barrier set-up and the TMEM allocation overlap that kernel's tail,
 // and nothing touches global memory before griddepcontrol.wait (measured
 // 42.3 -> 39.8 us per call at 16 tokens, 13.8 -> 12.8 us for the predictor
-// alone at 256).
+// alone at 256) -- except GEMM 2's producer and MMA warps, whose operands do not
+// depend on GEMM 1: up to 64 tokens the two GEMMs use 72 SMs each, so GEMM 2's
+// main loop runs beside GEMM 1 and only its epilogue waits (40.3 -> 37.4 us per
+// call at 16 tokens).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -91,6 +94,7 @@ struct GemmParams {
   uint16_t* out;          // GEMM 3 bf16 output [M][N] when split_k == 1
   DeviceControl* ctl;
   unsigned long long wait_limit_ns;
+  int early_main;         // GEMM 2: producer and MMA warps start before the kernel ahead completes
 };
 
 // ---------------------------------------------------------------- PTX wrappers
@@ -351,10 +355,18 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // The set-up above touches no global memory, so it may overlap the tail of the
-  // kernel ahead of this one on the stream (a programmatic launch); everything
-  // below runs once that kernel has completed and its writes are visible.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // kernel ahead of this one on the stream (a programmatic launch).  GEMM 2's
+  // operands (q[r:] and K2) do not depend on GEMM 1, which lets it launch only
+  // after its own wait: with early_main GEMM 2's producer and MMA warps start at
+  // once and only its epilogue waits (for GEMM 1's scores and moments).
+  // Otherwise everything below runs once the kernel ahead has completed and its
+  // writes are visible.
+  if (EPI == kEpiGate && p.early_main) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  } else {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
   if (tid == 0 && ld_relaxed_gpu(&ctl->abort)) *abort_flag = 1;
   __syncthreads();
 
@@ -491,6 +503,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
     const int quarter = warp & 3;  // TMEM lanes [32 quarter, 32 quarter + 32)
     const int row = quarter * 32 + lane;
     const int colgrp = (warp - 2) >> 2;  // gate epilogue: which quarter of the columns
+    if (EPI == kEpiGate && p.early_main) asm volatile("griddepcontrol.wait;" ::: "memory");
     uint32_t uses[2] = {0u, 0u};
     int acc = 0;
     for (int unit = blockIdx.x; unit < p.units; unit += gridDim.x) {
@@ -979,6 +992,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     g.theta = theta;
   }
+  g.early_main = 1;
   g.K = d2;
   g.nkb = (d2 + BK - 1) / BK;
   g.kb_per_split = g.nkb;
@@ -998,6 +1012,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   }
   if (e != cudaSuccess) return e;
   // GEMM 3: out = H_hi V + H_lo V
+  g.early_main = 0;
   g.N = d_model;
   g.K = d_ff;
   const bool wide3 = prefill_gemm3_wide(T, d_model, num_sms);
