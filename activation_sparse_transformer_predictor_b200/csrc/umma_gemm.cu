@@ -43,7 +43,7 @@
 // main loop runs beside GEMM 1 and only its epilogue waits (40.3 -> 37.4 us per
 // call at 16 tokens).  Where theta_kernel runs between them it is launched the
 // same way and releases GEMM 2 at once (T = 128 47.0 -> 42.8 us, T = 256 57.1 ->
-// 54.9).
+// 54.9); so does the split-K reduce behind GEMM 3 (T = 256 54.9 -> 53.3 us).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -779,6 +779,10 @@ __global__ void __launch_bounds__(128) theta_kernel(const float2* moments, int M
 
 // out = bf16(sum over splits, in split order) of the GEMM 3 partials.
 __global__ void splitk_reduce_kernel(const float* part, int splits, size_t n4, uint16_t* out) {
+  // launched programmatically behind GEMM 3: resident while it finishes, reads
+  // the partials once it has completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     float4 a = __ldcs(reinterpret_cast<const float4*>(part) + i);
@@ -1042,8 +1046,18 @@ cudaError_t launch_prefill(const PrefillArgs& a, int num_sms, cudaStream_t strea
   if (e != cudaSuccess) return e;
   if (splits > 1) {
     const size_t n4 = static_cast<size_t>(T) * d_model / 4;
-    splitk_reduce_kernel<<<num_sms * 4, 256, 0, stream>>>(part, splits, n4, static_cast<uint16_t*>(a.out));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(num_sms * 4);
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, static_cast<const float*>(part), splits, n4,
+                                static_cast<uint16_t*>(a.out))) != cudaSuccess)
+      return e;
   }
   return cudaSuccess;
 }
