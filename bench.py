@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle CPU baseline")
     ap.add_argument("--no-extra", action="store_true", help="skip the prefill / stat-topk extra lines")
-    ap.add_argument("--case", default=None, choices=["decode", "prefill", "predictor", "topk", "topk_causal",
+    ap.add_argument("--case", default=None, choices=["decode", "noalloc", "prefill", "predictor", "topk", "topk_causal",
                                                      "huber_bwd", "attention"],
                     help="profiling mode: run only this workload, plain launches (no graph), print per-call time")
     ap.add_argument("--tokens", type=int, default=256, help="--case prefill: tokens per call")
@@ -364,6 +364,23 @@ def run_case(args):
         gx = torch.empty_like(x)
         fn = lambda i: spark.stat_topk_huber_backward(x, g, k, 0.25, grad_x=gx)
         unit = f"Huber backward rows {rows} x {d}"
+    elif args.case == "noalloc":
+        # the single-launch fused kernel at one token, through the allocation-free entry point
+        from activation_sparse_transformer_predictor_b200 import _binding
+        w = synthetic.ffn_layer(D_MODEL, R, D_FF)
+        copies = [{n: t.to(dev) for n, t in w.items()}]
+        copies += [{n: t.clone() for n, t in copies[0].items()} for _ in range(3)]
+        q = synthetic.tokens(1, D_MODEL).to(dev)[0].contiguous()
+        out = torch.empty_like(q)
+        L = _binding.lib()
+
+        def fn(i):
+            c = copies[i % len(copies)]
+            rc = L.spark_ffn_forward_noalloc(q.data_ptr(), c["K1"].data_ptr(), c["K2"].data_ptr(), c["V"].data_ptr(),
+                                             D_MODEL, R, D_FF, K, out.data_ptr(), _binding.stream_handle())
+            if rc != 0:
+                raise _binding.SparkError("spark_ffn_forward_noalloc", rc)
+        unit = "no-allocation decode (fused kernel), T=1"
     elif args.case == "topk":
         rows, d, k = 8 * 4096, 4096, 256
         x = torch.randn(rows, d, device=dev, generator=torch.Generator(device=dev).manual_seed(5))
