@@ -283,3 +283,19 @@ def test_host_buffers_in_a_decode_loop_with_weight_overlap():
                 oh[i].zero_()
     finally:
         spark.set_weight_overlap(False)
+
+
+def test_host_buffers_unaligned_pinned_q_takes_the_copy_path():
+    """A pinned q_host that is not 16-byte aligned cannot be read by the first kernel in 16-byte chunks:
+    the call copies it with the copy engine instead, with the same bits."""
+    d_model, r, d_ff, k = GEMMA
+    dev, _ = make_layer(d_model, r, d_ff, 1, layer=130)
+    ref = spark.ffn_forward(dev["q"][0], dev["K1"], dev["K2"], dev["V"], k).cpu()
+    buf = torch.empty(d_model + 1, dtype=torch.bfloat16).pin_memory()
+    qh = buf[1:]
+    qh.copy_(dev["q"][0].cpu())
+    assert qh.data_ptr() % 16 != 0
+    out = spark.ffn_forward_host(qh, dev["K1"], dev["K2"], dev["V"], k)
+    torch.cuda.synchronize()
+    assert spark.query_status() == 0
+    assert torch.equal(out, ref)
