@@ -1,10 +1,13 @@
 /*
  * spark.h -- C ABI of libspark.so: the Spark FFN forward pass with statistical
- * top-k, and the standalone statistical top-k operator, on NVIDIA B200 (sm_100a).
+ * top-k, the standalone statistical top-k operator (plain, causally masked and
+ * Huber-smoothed with its gradient) and Spark Attention for one decoding
+ * position, on NVIDIA B200 (sm_100a).
  *
  * Method source: the paper-notes page "Spark Transformer: Reactivating Sparsity
  * in FFN and Attention" (NeurIPS 2025, arXiv 2506.06644), section 方法详解 /
- * 关键设计, items "Spark FFN" and "Statistical Top-k".  Notation follows it:
+ * 关键设计, items "Spark FFN", "Statistical Top-k" and "Spark Attention".
+ * Notation follows it:
  *
  *   x      = K1^T q[:r]                                   (low-rank predictor)
  *   theta  = mean(x) + std(x) * Q(1 - k/d_ff)             (Q: standard-normal quantile)
@@ -19,7 +22,8 @@
  *
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
- *     and must stay valid until the work enqueued on `stream` has finished.
+ *     and must stay valid until the work enqueued on `stream` has finished
+ *     (spark_ffn_forward_host alone takes q and out in host memory).
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream) and returns once the work is enqueued.  Argument errors
  *     are detected on the host before anything is enqueued.
