@@ -96,6 +96,7 @@ struct GemmParams {
   uint16_t* out;          // GEMM 3 bf16 output [M][N] when split_k == 1
   DeviceControl* ctl;
   unsigned long long wait_limit_ns;
+  int x_tma;              // predictor: X row-major through TMA stores (tensor map in the fourth map slot)
   int early_main;         // GEMM 2: producer and MMA warps start before the kernel ahead completes
 };
 
@@ -107,6 +108,17 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* tm, in
       "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
+
+// TMA store of a shared-memory box to a tensor-map region (bulk async group)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int c0, int c1, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(c0), "r"(c1), "r"(smem_u32(src))
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -549,15 +561,30 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
         constexpr int kEpiCols = kUC / 2;
         const int col0 = colgrp * kEpiCols;                 // first unit column of this warp
         const int tile0 = WIDE ? n_base + col0 : n_base;    // first column of its moments tile
-        float4* stg = reinterpret_cast<float4*>(smem + STAGES * kStageBytes + 256) + (warp - 2) * 256;
-        float* red = reinterpret_cast<float*>(smem + STAGES * kStageBytes + 256 + epi_warps(EPI) * 4096);
+        // staging blocks 1024-byte aligned (the TMA store reads them 128-byte swizzled)
+        float4* stg = reinterpret_cast<float4*>(smem + STAGES * kStageBytes + 1024) + (warp - 2) * 256;
+        float* red = reinterpret_cast<float*>(smem + STAGES * kStageBytes + 1024 + epi_warps(EPI) * 4096);
         float sum = 0.f;
 #pragma unroll 1
         for (int c = col0; c < col0 + kEpiCols; c += 32) {
           float w[32];
           tmem_ld32(taddr + c, w);
           const int nc0 = n_base + c;
-          if (p.X != nullptr) {
+          if (p.X != nullptr && p.x_tma) {
+            // lane l's 32 values go to row l of the warp's 32 x 32 staging block in the
+            // 128-byte-swizzled order (16-byte chunk j at j ^ (l % 8)); one lane then
+            // stores the block with one TMA instruction (rows >= M and columns >= N
+            // are clipped by the tensor map)
+            if (lane == 0) bulk_wait_read_all();  // the previous block has been read
+            __syncwarp();
+#pragma unroll
+            for (int q8 = 0; q8 < 8; ++q8)
+              stg[lane * 8 + (q8 ^ (lane & 7))] = make_float4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
+            fence_proxy_async_shared();
+            __syncwarp();
+            const int m0 = tm * BM + quarter * 32;
+            if (lane == 0 && m0 < p.M && nc0 < p.N) tma_store_2d(&tmB2, nc0, m0, stg);
+          } else if (p.X != nullptr) {
             // through shared memory: lane l's 32 values go to row l of a 32 x 32
             // staging block (16-byte chunks xor-swizzled by row), read back so that
             // one store instruction covers 4 rows x 128 contiguous bytes
@@ -723,6 +750,7 @@ __global__ void __launch_bounds__(gemm_threads(EPI), 1)
       ++uses[acc];
       acc ^= 1;
     }
+    if (EPI == kEpiPredictor && p.x_tma && lane == 0) bulk_wait_all();  // the TMA stores are done
   }
 
   // ------------------------------------------------------------ teardown
@@ -831,11 +859,25 @@ bool make_tmap(CUtensorMap* tm, const void* base, uint64_t inner, uint64_t outer
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [outer][inner] row-major, box (32 x 32), 128-byte swizzle: the predictor's X for TMA stores
+bool make_tmap_x(CUtensorMap* tm, void* base, uint64_t inner, uint64_t outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {inner * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 template <int EPI, bool B_NMAJOR, bool DUAL, int STAGES, bool WIDE = false, bool A64 = false, bool NW = false>
 cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& a2, const CUtensorMap& b, const CUtensorMap& b2,
                         const GemmParams& p, int num_sms, cudaStream_t stream) {
   constexpr int kStageBytes = (A64 ? kABytes / 2 : kABytes) * (DUAL ? 2 : 1) + (NW ? kBBytes / 2 : kBBytes) * (WIDE ? 2 : 1);
-  constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + 256 + (EPI == kEpiGate ? 8 * BM * 4 : 0) +
+  constexpr size_t smem = static_cast<size_t>(STAGES) * kStageBytes + 1024 + (EPI == kEpiPredictor ? 1024 : 256) +
+                          (EPI == kEpiGate ? 8 * BM * 4 : 0) +
                           (EPI == kEpiPredictor ? epi_warps(EPI) * 4096 + 2 * BM * 4 : 0);
   auto kern = umma_gemm_kernel<EPI, B_NMAJOR, DUAL, STAGES, WIDE, A64, NW>;
   static int set_dev = -1;
@@ -1073,13 +1115,15 @@ cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, 
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   const bool a64 = T <= 64;
   CUtensorMap tq1, tk1;
+  CUtensorMap tx;
   if (!make_tmap(&tq1, q, r, T, static_cast<uint64_t>(d_model) * 2, BK, a64 ? 64 : BM) ||
-      !make_tmap(&tk1, K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, BN))
+      !make_tmap(&tk1, K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, BN) || !make_tmap_x(&tx, x_out, d_ff, T))
     return cudaErrorInvalidValue;
   GemmParams g{};
   g.ctl = reinterpret_cast<DeviceControl*>(ws);
   g.wait_limit_ns = wait_limit_ns;
   g.X = x_out;
+  g.x_tma = 1;
   g.Xt = nullptr;
   g.xt_tiles_n = tiles_n;
   g.moments = nullptr;  // x only
@@ -1098,7 +1142,7 @@ cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, 
   if (wide_units >= num_sms) {
     g.tiles_n = (d_ff + 2 * BN - 1) / (2 * BN);
     g.units = wide_units;
-    return launch_gemm<kEpiPredictor, false, false, 4, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+    return launch_gemm<kEpiPredictor, false, false, 4, true>(tq1, tq1, tk1, tx, g, num_sms, stream);
   }
   if (T <= BM) {
     // one token band: 128 x 64 units, 144 CTAs streaming K1 (T = 16 10.8 -> 9.9 us,
@@ -1107,11 +1151,11 @@ cudaError_t launch_predictor(const void* q, const void* K1, int T, int d_model, 
     if (!make_tmap(&tk1n, K1, r, d_ff, static_cast<uint64_t>(r) * 2, BK, 64)) return cudaErrorInvalidValue;
     g.tiles_n = (d_ff + 63) / 64;
     g.units = g.tiles_m * g.tiles_n;
-    return a64 ? launch_gemm<kEpiPredictor, false, false, 12, false, true, true>(tq1, tq1, tk1n, tk1n, g, num_sms, stream)
-               : launch_gemm<kEpiPredictor, false, false, 8, false, false, true>(tq1, tq1, tk1n, tk1n, g, num_sms, stream);
+    return a64 ? launch_gemm<kEpiPredictor, false, false, 12, false, true, true>(tq1, tq1, tk1n, tx, g, num_sms, stream)
+               : launch_gemm<kEpiPredictor, false, false, 8, false, false, true>(tq1, tq1, tk1n, tx, g, num_sms, stream);
   }
-  if (a64) return launch_gemm<kEpiPredictor, false, false, 8, false, true>(tq1, tq1, tk1, tk1, g, num_sms, stream);
-  return launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tk1, g, num_sms, stream);
+  if (a64) return launch_gemm<kEpiPredictor, false, false, 8, false, true>(tq1, tq1, tk1, tx, g, num_sms, stream);
+  return launch_gemm<kEpiPredictor, false, false, 6>(tq1, tq1, tk1, tx, g, num_sms, stream);
 }
 
 
