@@ -4,7 +4,7 @@
 // tokens at once:
 //   GEMM 1  X = Q1 K1^T                 (predictor; x = K1^T q[:r] per token)
 //           epilogue: x stored once, fp32, in 128 x 128 tiles, and the
-//           per-(token, 128-neuron tile) moments of x
+//           per-(token, 128- or 64-neuron tile) moments of x
 //   GEMM 2  A = Q2 K2^T
 //           epilogue: theta per token from the tile moments, theta = mean +
 //           std Q(1 - k/d_ff) (merged by the epilogue warps while the main loop
@@ -33,17 +33,20 @@
 // that the epilogue of one tile overlaps the main loop of the next), the
 // remaining warps = epilogue (tcgen05.ld, 32 TMEM lanes per warp).  A unit is
 // 128 tokens x 128 columns, x 256 once there are enough to fill the SMs, or x 64
-// for GEMMs 1 and 2 with a single token band (more CTAs streaming the weights).  Every wait
-// is bounded.  Each GEMM is launched as a programmatic dependent of the kernel
-// before it: barrier set-up and the TMEM allocation overlap that kernel's tail,
-// and nothing touches global memory before griddepcontrol.wait (measured
-// 42.3 -> 39.8 us per call at 16 tokens, 13.8 -> 12.8 us for the predictor
-// alone at 256) -- except GEMM 2's producer and MMA warps, whose operands do not
-// depend on GEMM 1: up to 64 tokens the two GEMMs use 72 SMs each, so GEMM 2's
-// main loop runs beside GEMM 1 and only its epilogue waits (40.3 -> 37.4 us per
-// call at 16 tokens).  Where theta_kernel runs between them it is launched the
-// same way and releases GEMM 2 at once (T = 128 47.0 -> 42.8 us, T = 256 57.1 ->
-// 54.9); so does the split-K reduce behind GEMM 3 (T = 256 54.9 -> 53.3 us).
+// for GEMMs 1 and 2 with a single band of 65-128 tokens (more CTAs streaming the
+// weights).  The predictor entry point writes x row-major by TMA tensor stores.
+// Every wait is bounded.
+//
+// Each GEMM is launched as a programmatic dependent of the kernel before it:
+// barrier set-up and the TMEM allocation overlap that kernel's tail, and nothing
+// touches global memory before griddepcontrol.wait (measured 42.3 -> 39.8 us per
+// call at 16 tokens, 13.8 -> 12.8 us for the predictor alone at 256) -- except
+// GEMM 2's producer and MMA warps, whose operands do not depend on GEMM 1: up to
+// 64 tokens the two GEMMs use 72 SMs each, so GEMM 2's main loop runs beside
+// GEMM 1 and only its epilogue waits (40.3 -> 37.4 us per call at 16 tokens).
+// Where theta_kernel runs between them it is launched the same way and releases
+// GEMM 2 at once (T = 128 47.0 -> 42.8 us, T = 256 57.1 -> 54.9); so does the
+// split-K reduce behind GEMM 3 (T = 256 54.9 -> 53.3 us).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
