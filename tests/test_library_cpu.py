@@ -127,3 +127,22 @@ def test_debug_library_exports_the_same_symbols(L):
         assert hasattr(D, name), name
     assert D.spark_version() == L.spark_version()
     assert L.spark_debug_violations() == -1
+
+
+def test_using_library_routes_every_wrapper_and_restores(L):
+    """The binding's override (used to run the wrappers through the bounds-checked
+    build) applies inside the block only, and nests."""
+    D = _binding.debug_lib()
+    assert _binding.lib() is L
+    with _binding.using_library(D):
+        assert _binding.lib() is D
+        with _binding.using_library(L):
+            assert _binding.lib() is L
+        assert _binding.lib() is D
+    assert _binding.lib() is L
+    try:
+        with _binding.using_library(D):
+            raise KeyError("inside")
+    except KeyError:
+        pass
+    assert _binding.lib() is L
