@@ -146,3 +146,50 @@ def test_using_library_routes_every_wrapper_and_restores(L):
     except KeyError:
         pass
     assert _binding.lib() is L
+
+
+def _strip_comments(src):
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    return re.sub(r"//[^\n]*", " ", src)
+
+
+def _function_body(src, signature):
+    """The text between the braces of the function whose definition starts with
+    `signature` (brace matching on comment-free source)."""
+    start = src.index(signature)
+    i = src.index("{", start)
+    depth = 0
+    for j in range(i, len(src)):
+        depth += {"{": 1, "}": -1}.get(src[j], 0)
+        if depth == 0:
+            return src[i:j + 1]
+    raise AssertionError("unbalanced braces after " + signature)
+
+
+ALLOCATING = re.compile(r"\b(cudaMalloc\w*|cudaHostAlloc|cudaMemPool\w*|cuMem\w*|get_buffer|get_workspace|"
+                        r"ffn_forward_impl|malloc|calloc|realloc)\b|\bnew\s+[\w:]")
+
+
+def test_noalloc_entry_point_names_no_allocator():
+    """spark_ffn_forward_noalloc's defining property, checked on its source: its
+    translation unit and the fused launcher it calls name no device, host or pool
+    allocator and do not reach the workspace pool that the other entry points grow."""
+    csrc = os.path.join(ROOT, "activation_sparse_transformer_predictor_b200", "csrc")
+    noalloc = _strip_comments(open(os.path.join(csrc, "spark_noalloc.cu")).read())
+    assert "launch_fused(" in noalloc
+    assert not ALLOCATING.search(noalloc), ALLOCATING.search(noalloc).group(0)
+    fused = _strip_comments(open(os.path.join(csrc, "ffn_fused.cu")).read())
+    api = _strip_comments(open(os.path.join(csrc, "spark_api.cu")).read())
+    body = _function_body(fused, "cudaError_t launch_fused(const FusedPlan&")
+    assert "cudaLaunchKernelEx" in body
+    # the host helpers it calls: the launch plan, k's quantile, the wait limit
+    for name in ("plan_fused", "spark_topk_quantile", "wait_limit_ns"):
+        assert name + "(" in noalloc, name
+    body += _function_body(fused, "FusedPlan plan_fused(")
+    body += _function_body(api, "double spark_topk_quantile(int k, int d)")
+    body += _function_body(api, "double upper_tail_quantile(")
+    body += _function_body(api, "unsigned long long wait_limit_ns()")
+    assert not ALLOCATING.search(body), ALLOCATING.search(body).group(0)
+    # the pattern does catch what it is meant to catch
+    for bad in ("cudaMallocAsync(&p, n, s)", "get_buffer(pool, dev, s, n, true, &p)", "auto* p = new float[4];"):
+        assert ALLOCATING.search(bad), bad
