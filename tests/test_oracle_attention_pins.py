@@ -133,3 +133,35 @@ def test_brute_force_tiny():
     res = oracle.spark_attention(q, K, V, r, k_attn=k, scale=scale)
     assert res["theta"][0] == pytest.approx(theta, rel=1e-13)
     np.testing.assert_allclose(res["out"][0], expect, rtol=1e-12, atol=1e-14)
+
+
+def test_override_set_renormalises_over_the_given_keys():
+    """override_active replaces the selected set A: the softmax weights are renormalised over the given
+    keys (checked against a plain numpy evaluation), an empty set gives 0, A itself gives the plain
+    result, and the reported mask stays the predictor's own (s > theta)."""
+    n_heads, n_kv, n_ctx, d_head, r, k = 4, 2, 40, 16, 8, 6
+    q, K, V = make(n_heads, n_kv, n_ctx, d_head, 31)
+    base = oracle.spark_attention(q, K, V, r, k_attn=k, scale=0.5)
+    same = oracle.spark_attention(q, K, V, r, k_attn=k, scale=0.5, override_active=base["active"])
+    assert np.array_equal(same["out"], base["out"]) and np.array_equal(same["active"], base["active"])
+    none = oracle.spark_attention(q, K, V, r, k_attn=k, scale=0.5,
+                                  override_active=np.zeros((n_heads, n_ctx), bool))
+    assert np.all(none["out"] == 0.0) and np.array_equal(none["active"], base["active"])
+    # a different set: drop each head's first selected key, add its two highest unselected ones
+    ov = base["active"].copy()
+    for h in range(n_heads):
+        on = np.flatnonzero(ov[h])
+        off = np.flatnonzero(~ov[h])
+        ov[h, on[0]] = False
+        ov[h, off[np.argsort(base["s"][h, off])[-2:]]] = True
+    res = oracle.spark_attention(q, K, V, r, k_attn=k, scale=0.5, override_active=ov)
+    assert np.array_equal(res["active"], base["active"])
+    qf, Kf, Vf = widen(q), widen(K), widen(V)
+    for h in range(n_heads):
+        g = h // (n_heads // n_kv)
+        sel = np.flatnonzero(ov[h])
+        s = 0.5 * (Kf[g, sel, :r] @ qf[h, :r])
+        p = np.exp(s - s.max()) / np.exp(s - s.max()).sum()
+        a = Kf[g, sel, r:] @ qf[h, r:]
+        expect = (p * np.log1p(np.exp(a))) @ Vf[g, sel]
+        np.testing.assert_allclose(res["out"][h], expect, rtol=1e-12, atol=1e-14)

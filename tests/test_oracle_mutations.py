@@ -29,6 +29,16 @@ MUTATIONS = {
     "gelu_of_x_not_s": ("double g = gelu_of_kind(s, gelu_kind);", "double g = gelu_of_kind(x[i], gelu_kind);"),
     "drops_a": ("double h = g * a;", "double h = g;"),
     "soft_threshold_not_clamped": ("out[row * d + i] = s > 0.0 ? s : 0.0;", "out[row * d + i] = s;"),
+    "mean_wrong_divisor": ("double mean = sum / (double)d;", "double mean = sum / (double)(d - 1);"),
+    "gelu_half_dropped": ("return 0.5 * s * (1.0 + tanh(", "return s * (1.0 + tanh("),
+    "gelu_one_dropped": ("(1.0 + tanh(c * (s", "(tanh(c * (s"),
+    "quantile_tail_complement": ("double tail = k / d;", "double tail = 1.0 - k / d;"),
+    "gelu_erf_sign": ("s * 0.5 * erfc(-s / sqrt(2.0))", "s * 0.5 * erfc(s / sqrt(2.0))"),
+    "rmsnorm_eps_dropped": ("1.0 / sqrt(ss / (double)d + eps);", "1.0 / sqrt(ss / (double)d);"),
+    "rmsnorm_sum_not_mean": ("1.0 / sqrt(ss / (double)d + eps);", "1.0 / sqrt(ss + eps);"),
+    "ffn_override_unclamped": ("            if (s < 0.0) s = 0.0;\n            double g = gelu_of_kind", "            double g = gelu_of_kind"),
+    "ffn_mask_from_override": ("if (active_out) active_out[t * d_ff + i] = (uint8_t)(x[i] > theta);",
+                               "if (active_out) active_out[t * d_ff + i] = (uint8_t)active;"),
 }
 
 
@@ -45,6 +55,12 @@ ATTN_MUTATIONS = {
     "attn_theta_ignored": ("if (k_attn < n_ctx) theta = oracle_theta(s, n_ctx, k_attn, NULL, NULL);", ""),
     "attn_value_from_key": ("o[c] += f * oracle_bf16_to_f64(Vg[j * d_head + c]);",
                             "o[c] += f * oracle_bf16_to_f64(Kg[j * d_head + c]);"),
+    "attn_softmax_over_all_keys": ("            if (!act) continue;\n            double w = exp(s[j] - smax);",
+                                   "            double w = exp(s[j] - smax);\n            if (!act) { z += w; continue; }"),
+    "attn_softplus_to_identity": ("double f = w * oracle_softplus(a);", "double f = w * a;"),
+    "attn_theta_at_k_equal_n": ("if (k_attn < n_ctx) theta", "if (k_attn <= n_ctx) theta"),
+    "attn_mask_from_override": ("if (active_out) active_out[h * n_ctx + j] = (uint8_t)(s[j] > theta);",
+                                "if (active_out) active_out[h * n_ctx + j] = (uint8_t)act;"),
 }
 
 
@@ -58,6 +74,10 @@ CAUSAL_MUTATIONS = {
     "causal_select_all_zeroed": ("for (long j = 0; j < n; ++j) out[row * d + j] = xr[j];",
                                  "for (long j = 0; j < n; ++j) out[row * d + j] = 0.0;"),
     "causal_select_all_boundary": ("        if (k < n) {\n            double mean, sd;", "        if (k <= n) {\n            double mean, sd;"),
+    "causal_theta_misses_last_visible": ("theta = oracle_theta(xr, n, k, &mean, &sd);",
+                                         "theta = oracle_theta(xr, n > 1 ? n - 1 : n, k, &mean, &sd);"),
+    "causal_pass_through_clamped": ("for (long j = 0; j < n; ++j) out[row * d + j] = xr[j];",
+                                    "for (long j = 0; j < n; ++j) out[row * d + j] = xr[j] > 0.0 ? xr[j] : 0.0;"),
 }
 
 
@@ -70,6 +90,7 @@ HUBER_MUTATIONS = {
     "huber_middle_slope": ("if (z < delta) return z / delta;", "if (z < delta) return z / (2.0 * delta);"),
     "huber_forward_offset": ("return z - 0.5 * delta;", "return z - delta;"),
     "huber_forward_square": ("if (z < delta) return z * z / (2.0 * delta);", "if (z < delta) return z * z / delta;"),
+    "huber_backward_drops_mean_term": ("double dtheta = 1.0 / (double)d;", "double dtheta = 0.0;"),
 }
 
 

@@ -302,6 +302,7 @@ def test_ffn_override_active_set():
     assert np.array_equal(same["out"], base["out"])
     none = oracle.spark_ffn(q, K1, K2, V, r, k, override_active=np.zeros((T, d_ff), bool))
     assert np.all(none["out"] == 0)
+    assert np.array_equal(none["active"], base["active"])  # the reported mask stays x > theta
     # every neuron "active": inactive ones have max(x - theta, 0) = 0 and GELU(0) = 0
     allon = oracle.spark_ffn(q, K1, K2, V, r, k, override_active=np.ones((T, d_ff), bool))
     np.testing.assert_allclose(allon["out"], base["out"], rtol=0, atol=1e-14)
