@@ -334,16 +334,15 @@ SPARK_API int spark_selftest_wait_timeout(spark_stream_t stream);
  *
  * Set-up: the first call on a device looks up the buffer's device address
  * (cudaGetSymbolAddress) with that device current and keeps it for the rest of
- * the process; make that first call before any stream capture.  A
- * cudaDeviceReset (or any reset of the device's primary context) unmaps the
+ * the process.  A cudaDeviceReset (or any reset of the device's primary context) unmaps the
  * buffer and leaves that address stale: do not call this entry point on a
  * device after resetting it.
  *
  * Sharing: all calls on all streams use the same buffer, which keeps the last
  * call's contents.  Each call clears the buffer's arrival counters with a
  * cudaMemsetAsync on `stream` before its kernel.  Calls whose work overlaps on
- * the GPU (on different streams, or in graphs replayed concurrently) race on
- * the buffer and give wrong results: order them.
+ * the GPU (on different streams) race on the buffer and give wrong results:
+ * order them.
  *
  * Errors: every device-side wait has the time limit of spark_set_wait_limit_ns.
  * A wait that runs out leaves `out` undefined and records SPARK_ETIMEOUT in the
